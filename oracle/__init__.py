@@ -1,0 +1,276 @@
+"""CPU oracle for group-wise RTN weight quantization and the W4A16 linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The product path
+(``w4a16_bit_gemm_b200``) never imports it and shares no code with it.
+
+The arithmetic lives in ``wq_oracle.c`` (plain C, fp32/fp64 with explicit
+IEEE 754 conversions written from the standard); this module only builds the
+shared object with gcc and marshals numpy arrays through ctypes.
+
+Source pages (title, section):
+  * "LLM Quantization: GPTQ, AWQ, SmoothQuant, FP8, KV Cache (7/10)",
+    blog.ruahverce.com: "Affine Quantization", "Symmetric and Asymmetric",
+    "Per-group", "Memory arithmetic", "Group scale overhead".
+  * "Quantization Algorithms" (V10 study notes), brianyu43.github.io:
+    section 1.8 "Signed vs Unsigned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+FLAG_NONFINITE = 1
+FLAG_RANGE = 2
+
+
+def _compile(out: str, mutant: int = 0) -> None:
+    tmp = out + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+           "-fno-fast-math", "-pthread", "-DWQO_MUTANT=%d" % mutant, _SRC, "-o", tmp, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, out)
+
+
+def build(force: bool = False) -> str:
+    """Compile ``wq_oracle.c`` into ``liboracle.so`` next to it (gcc, -O2,
+    strict IEEE: no -ffast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        _compile(_LIB, 0)
+    return _LIB
+
+
+def build_mutant(mutant: int, out_dir: str) -> str:
+    """Build a copy of the oracle with one planted mistake (test use only)."""
+    out = os.path.join(out_dir, "liboracle_mutant%d.so" % mutant)
+    _compile(out, mutant)
+    return out
+
+
+class use_library:
+    """Context manager that routes this module's calls to another build of
+    the oracle (a planted-mistake variant) and restores the real one."""
+
+    def __init__(self, path: str):
+        self.path = path
+        self.saved = None
+
+    def __enter__(self):
+        global _lib
+        _load()
+        self.saved = _lib
+        _lib = None
+        _load(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
+
+
+def _load(path: str | None = None):
+    global _lib
+    with _lock:
+        if _lib is None:
+            if path is None:
+                build()
+            lib = ctypes.CDLL(path or _LIB)
+            P = ctypes.c_void_p
+            i64 = ctypes.c_int64
+            i32 = ctypes.c_int
+            lib.wqo_quantize.argtypes = [P, i64, i64, i64, i32, i32, i32, P, P, P, P, i32]
+            lib.wqo_quantize.restype = i32
+            lib.wqo_pack4.argtypes = [P, i64, i64, P]
+            lib.wqo_pack4.restype = i32
+            lib.wqo_unpack4.argtypes = [P, i64, i64, i32, P]
+            lib.wqo_unpack4.restype = i32
+            lib.wqo_dequantize.argtypes = [P, P, P, i64, i64, i64, P, i32]
+            lib.wqo_dequantize.restype = i32
+            lib.wqo_linear.argtypes = [P, i64, P, i64, i64, P, P, i32]
+            lib.wqo_linear.restype = i32
+            lib.wqo_artifact_bytes.argtypes = [i64, i32, i64, i32, P, P, P]
+            lib.wqo_artifact_bytes.restype = i32
+            lib.wqo_f32_to_bf16.argtypes = [ctypes.c_float]
+            lib.wqo_f32_to_bf16.restype = ctypes.c_uint16
+            lib.wqo_f32_to_f16.argtypes = [ctypes.c_float]
+            lib.wqo_f32_to_f16.restype = ctypes.c_uint16
+            lib.wqo_f16_to_f32.argtypes = [ctypes.c_uint16]
+            lib.wqo_f16_to_f32.restype = ctypes.c_float
+            lib.wqo_bf16_to_f32.argtypes = [ctypes.c_uint16]
+            lib.wqo_bf16_to_f32.restype = ctypes.c_float
+            lib.wqo_dequant_one.argtypes = [ctypes.c_uint16, ctypes.c_int32, ctypes.c_int32]
+            lib.wqo_dequant_one.restype = ctypes.c_uint16
+            for nm in ("wqo_f32_to_f16_array", "wqo_f32_to_bf16_array", "wqo_f16_to_f32_array"):
+                getattr(lib, nm).argtypes = [P, i64, P]
+                getattr(lib, nm).restype = None
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------------------
+# scalar conversions (exposed for pins)
+# --------------------------------------------------------------------------
+
+def f32_to_bf16_bits(x: float) -> int:
+    return int(_load().wqo_f32_to_bf16(float(x)))
+
+
+def f32_to_f16_bits(x: float) -> int:
+    return int(_load().wqo_f32_to_f16(float(x)))
+
+
+def f16_bits_to_f32(h: int) -> float:
+    return float(_load().wqo_f16_to_f32(int(h)))
+
+
+def bf16_bits_to_f32(h: int) -> float:
+    return float(_load().wqo_bf16_to_f32(int(h)))
+
+
+def dequant_one(s16: int, q: int, z: int) -> int:
+    return int(_load().wqo_dequant_one(int(s16), int(q), int(z)))
+
+
+def f32_to_f16_bits_array(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint16)
+    _load().wqo_f32_to_f16_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def f32_to_bf16_bits_array(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint16)
+    _load().wqo_f32_to_bf16_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def f16_bits_to_f32_array(h: np.ndarray) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(h.shape, np.float32)
+    _load().wqo_f16_to_f32_array(_ptr(h), h.size, _ptr(out))
+    return out
+
+
+# --------------------------------------------------------------------------
+# array operations; bf16/fp16 tensors are carried as uint16 bit patterns
+# --------------------------------------------------------------------------
+
+def quantize(W_bits: np.ndarray, group_size: int, bits: int = 4, symmetric: bool = False,
+             narrow: bool = False, nthreads: int | None = None):
+    """Group-wise RTN quantization of bf16 weights ``W_bits`` (uint16 [d_out, d_in]).
+
+    Returns ``(codes int32 [d_out,d_in], scales uint16 [d_out,G], zeros uint16
+    [d_out,G] or None, flags)``.
+    """
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    d_out, d_in = W_bits.shape
+    G = d_in // group_size
+    codes = np.empty((d_out, d_in), np.int32)
+    scales = np.empty((d_out, G), np.uint16)
+    zeros = None if symmetric else np.empty((d_out, G), np.uint16)
+    flags = ctypes.c_uint32(0)
+    rc = _load().wqo_quantize(_ptr(W_bits), d_out, d_in, group_size, bits, int(symmetric),
+                              int(narrow), _ptr(codes), _ptr(scales),
+                              _ptr(zeros) if zeros is not None else None,
+                              ctypes.cast(ctypes.pointer(flags), ctypes.c_void_p),
+                              nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle quantize rejected its arguments")
+    return codes, scales, zeros, int(flags.value)
+
+
+def pack4(codes: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.int32)
+    d_out, d_in = codes.shape
+    q = np.empty((d_out, d_in // 8), np.uint32)
+    if _load().wqo_pack4(_ptr(codes), d_out, d_in, _ptr(q)) != 0:
+        raise ValueError("oracle pack4 rejected its arguments")
+    return q
+
+
+def unpack4(qweight: np.ndarray, d_in: int, symmetric: bool) -> np.ndarray:
+    qweight = np.ascontiguousarray(qweight, dtype=np.uint32)
+    d_out = qweight.shape[0]
+    codes = np.empty((d_out, d_in), np.int32)
+    if _load().wqo_unpack4(_ptr(qweight), d_out, d_in, int(symmetric), _ptr(codes)) != 0:
+        raise ValueError("oracle unpack4 rejected its arguments")
+    return codes
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, zeros, group_size: int,
+               nthreads: int | None = None) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.int32)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    d_out, d_in = codes.shape
+    out = np.empty((d_out, d_in), np.uint16)
+    zp = None
+    if zeros is not None:
+        zeros = np.ascontiguousarray(zeros, dtype=np.uint16)
+        zp = _ptr(zeros)
+    if _load().wqo_dequantize(_ptr(codes), _ptr(scales), zp, d_out, d_in, group_size,
+                              _ptr(out), nthreads or default_threads()) != 0:
+        raise ValueError("oracle dequantize rejected its arguments")
+    return out
+
+
+def linear(X_bits: np.ndarray, W_hat_bits: np.ndarray, nthreads: int | None = None):
+    """fp64 ``Y[m,n] = sum_k W_hat[n,k] X[m,k]`` and ``A[m,n] = sum_k |W_hat X|``."""
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    W_hat_bits = np.ascontiguousarray(W_hat_bits, dtype=np.uint16)
+    M, K = X_bits.shape
+    N, K2 = W_hat_bits.shape
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    Y = np.empty((M, N), np.float64)
+    A = np.empty((M, N), np.float64)
+    if _load().wqo_linear(_ptr(X_bits), M, _ptr(W_hat_bits), N, K, _ptr(Y), _ptr(A),
+                          nthreads or default_threads()) != 0:
+        raise ValueError("oracle linear rejected its arguments")
+    return Y, A
+
+
+def artifact_bytes(params: int, bits: int, group_size: int, symmetric: bool):
+    """(payload, scale bytes, zero bytes) of a packed artifact."""
+    p, s, z = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    _load().wqo_artifact_bytes(int(params), int(bits), int(group_size), int(symmetric),
+                               ctypes.cast(ctypes.pointer(p), ctypes.c_void_p),
+                               ctypes.cast(ctypes.pointer(s), ctypes.c_void_p),
+                               ctypes.cast(ctypes.pointer(z), ctypes.c_void_p))
+    return p.value, s.value, z.value
+
+
+def quantize_pack4(W_bits: np.ndarray, group_size: int = 128, symmetric: bool = False,
+                   nthreads: int | None = None):
+    """4-bit quantize + pack: ``(qweight uint32 [d_out,d_in/8], scales, zeros, flags, codes)``."""
+    codes, scales, zeros, flags = quantize(W_bits, group_size, 4, symmetric, False, nthreads)
+    return pack4(codes), scales, zeros, flags, codes
+
+
+def reference_linear_w4a16(X_bits, W_bits, group_size=128, symmetric=False, nthreads=None):
+    """Whole path on the CPU: quantize, dequantize, fp64 linear.  Returns
+    ``(Y, A, W_hat_bits, (qweight, scales, zeros, flags))``."""
+    qweight, scales, zeros, flags, codes = quantize_pack4(W_bits, group_size, symmetric, nthreads)
+    W_hat = dequantize(codes, scales, zeros, group_size, nthreads)
+    Y, A = linear(X_bits, W_hat, nthreads)
+    return Y, A, W_hat, (qweight, scales, zeros, flags)

@@ -1,0 +1,499 @@
+/*
+ * wq_oracle.c -- plain, slow, obviously-correct CPU oracle for group-wise RTN
+ * affine weight quantization, dequantization and the W4A16 linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA path and includes no CUDA header.
+ *
+ * Sources (page title, section):
+ *  [P1] "LLM Quantization: GPTQ, AWQ, SmoothQuant, FP8, KV Cache (7/10)",
+ *       blog.ruahverce.com -- sections "Affine Quantization", "Bit count and
+ *       level count", "Symmetric and Asymmetric", "Per-group", "Memory
+ *       arithmetic: payload and metadata", "Group scale overhead",
+ *       "Fused low-bit kernel (path A) / full dequantize then matmul (path B)".
+ *  [P2] "Quantization Algorithms" (V10 study notes), brianyu43.github.io --
+ *       section 1.8 "Signed vs Unsigned" (INT8 symmetric uses [-127,127],
+ *       INT4 signed [-8,7], asymmetric unsigned [0,15]); "Fake vs real quant"
+ *       section 4 (dequantized value multiplied in floating point, one
+ *       rounding).
+ *
+ * What is computed (each step in the order the pages give it):
+ *   quantize  q = clamp(round(x / s) + z, q_min, q_max)          [P1 Affine]
+ *   symmetric z = 0, s = max|x| / q_max                          [P1 Symmetric]
+ *   asymmetric s = (x_max - x_min) / (q_max - q_min),
+ *              z = q_min - x_min / s, rounded and clamped so that
+ *              zero is exactly representable                     [P1 Asymmetric]
+ *   dequantize x_hat = s (q - z)                                 [P1 Affine]
+ *   linear     y[m,n] = sum_k x_hat[n,k] * x[m,k]                [P1 path A/B]
+ *
+ * Readings taken where the pages are silent (each is listed in the design
+ * notes of the repository):
+ *   - round() is round-half-to-even, applied to the IEEE fp32 quotient x/s;
+ *   - the quotient uses the STORED fp16 scale, so codes and dequant agree;
+ *   - the asymmetric range is widened to contain 0 (x_min' = min(0, min x),
+ *     x_max' = max(0, max x)) and z is an integer in [q_min, q_max]; then
+ *     code z dequantizes to exactly 0;
+ *   - s is computed in fp32 ((x_max' - x_min') / q_range, IEEE divide) and
+ *     rounded to fp16 with round-to-nearest-even; a zero fp16 scale (all-zero
+ *     or underflowing group) is replaced by s = 1, z = 0; an fp16 overflow
+ *     saturates s to 65504 and raises WQO_FLAG_RANGE;
+ *   - NaN inputs are skipped by the statistics and coded as the code of zero
+ *     (q = z); any NaN/Inf input raises WQO_FLAG_NONFINITE;
+ *   - symmetric 4-bit codes are stored as 4-bit two's complement nibbles;
+ *   - packing: 8 nibbles per uint32, nibble j of word c holds column 8c+j
+ *     (bits 4j..4j+3, low nibble first); scales/zeros are fp16 [d_out][d_in/g].
+ *
+ * Floating-point conversions are written here from the IEEE 754 definitions
+ * (binary32 -> binary16 and binary32 -> bfloat16, round to nearest even,
+ * subnormals included); nothing is taken from a vendor library.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* WQO_MUTANT (default 0) plants one deliberate mistake; the test suite
+ * builds each mutant separately to show that the pins catch it.  The
+ * shipped oracle is always built with WQO_MUTANT == 0. */
+#ifndef WQO_MUTANT
+#define WQO_MUTANT 0
+#endif
+
+#define WQO_FLAG_NONFINITE 1u
+#define WQO_FLAG_RANGE 2u
+
+/* ------------------------------------------------------------------------ */
+/* IEEE 754 conversions                                                      */
+/* ------------------------------------------------------------------------ */
+
+static float bits_to_f32(uint32_t u) {
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+static uint32_t f32_to_bits(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return u;
+}
+
+/* bfloat16 is the upper half of a binary32: widening is exact. */
+float wqo_bf16_to_f32(uint16_t h) { return bits_to_f32((uint32_t)h << 16); }
+
+/* binary32 -> bfloat16, round to nearest, ties to even.  The discarded low
+ * 16 bits are compared with one half of the bf16 unit in the last place. */
+uint16_t wqo_f32_to_bf16(float f) {
+    uint32_t u = f32_to_bits(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) /* NaN: keep sign, force quiet */
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t kept = u >> 16;
+    uint32_t dropped = u & 0xffffu;
+    if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u)))
+        kept += 1u; /* a carry into the exponent gives the next binade / inf */
+    return (uint16_t)kept;
+}
+
+/* binary16 -> binary32, exact. */
+float wqo_f16_to_f32(uint16_t h) {
+    uint32_t sign = (uint32_t)(h & 0x8000u) << 16;
+    uint32_t e = (h >> 10) & 0x1fu;
+    uint32_t m = h & 0x3ffu;
+    if (e == 0x1fu) return bits_to_f32(sign | 0x7f800000u | (m << 13));
+    if (e == 0) { /* zero or subnormal: m * 2^-24 */
+        float v = (float)m * 0x1p-24f;
+        return sign ? -v : v;
+    }
+    return bits_to_f32(sign | ((e - 15u + 127u) << 23) | (m << 13));
+}
+
+/* binary32 -> binary16, round to nearest, ties to even, with subnormals and
+ * overflow to infinity.  Let the input be mant * 2^(e-23) with a 24-bit
+ * integer significand.  The binary16 quantum at that magnitude is
+ * 2^(max(e,-14) - 10); the number of quanta is mant >> sh with
+ * sh = 13 + (max(e,-14) - e), rounded to nearest even on the dropped bits.
+ * The encoding ((E + 14) << 10) + q is valid for normals and subnormals and
+ * carries naturally into the next binade. */
+uint16_t wqo_f32_to_f16(float f) {
+    uint32_t u = f32_to_bits(f);
+    uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    uint32_t a = u & 0x7fffffffu;
+    if (a > 0x7f800000u) return (uint16_t)(sign | 0x7e00u); /* NaN */
+    if (a == 0x7f800000u) return (uint16_t)(sign | 0x7c00u); /* inf */
+    int e;
+    uint32_t mant;
+    if (a >= 0x00800000u) {
+        e = (int)(a >> 23) - 127;
+        mant = (a & 0x7fffffu) | 0x800000u;
+    } else {
+        e = -126;
+        mant = a;
+    }
+    int E = e > -14 ? e : -14;
+    int sh = 13 + (E - e);
+    uint32_t q;
+    if (sh >= 25) {
+        q = 0; /* below half of the smallest subnormal */
+    } else {
+        q = mant >> sh;
+        uint32_t rem = mant & ((1u << sh) - 1u);
+        uint32_t half = 1u << (sh - 1);
+        if (rem > half || (rem == half && (q & 1u))) q += 1u;
+    }
+    int64_t bits = ((int64_t)(E + 14) << 10) + (int64_t)q;
+    if (bits >= 0x7c00) return (uint16_t)(sign | 0x7c00u);
+    return (uint16_t)(sign | (uint16_t)bits);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantization parameters                                                   */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int bits;       /* b: 2, 4 or 8 */
+    int symmetric;  /* 1: z = 0, signed codes */
+    int narrow;     /* symmetric only: q_min = -q_max (INT8 [-127,127]) */
+} wqo_qparams;
+
+/* Code range: unsigned b bits give 2^b levels [0, 2^b - 1]; signed b bits
+ * give [-2^(b-1), 2^(b-1) - 1], and the narrow symmetric form drops the
+ * negative endpoint ([P1 Bit count and level count], [P2 1.8]). */
+static void code_range(const wqo_qparams* p, int* qmin, int* qmax) {
+    if (p->symmetric) {
+        *qmax = (1 << (p->bits - 1)) - 1;
+        *qmin = p->narrow ? -*qmax : -(1 << (p->bits - 1));
+    } else {
+        *qmin = 0;
+        *qmax = (1 << p->bits) - 1;
+    }
+}
+
+/* Clamp with IEEE maxNum/minNum semantics, then convert the (integral)
+ * float to int.  Inputs here are never NaN. */
+static int clamp_to_int(float v, int lo, int hi) {
+    if (v < (float)lo) v = (float)lo;
+    if (v > (float)hi) v = (float)hi;
+    return (int)v;
+}
+
+/* One group: derive (s, z) and the codes of g consecutive weights of one row.
+ * x: g bf16 words; codes: g ints; returns flags. */
+static uint32_t quantize_group(const uint16_t* x, int64_t g, const wqo_qparams* p,
+                               int32_t* codes, uint16_t* s_out, uint16_t* z_out) {
+    int qmin, qmax;
+    code_range(p, &qmin, &qmax);
+    uint32_t flags = 0;
+
+    /* statistics [P1 Symmetric / Asymmetric]; range widened to contain 0 */
+    float lo = 0.0f, hi = 0.0f, amax = 0.0f;
+#if WQO_MUTANT == 4 /* mistake: range not widened to contain zero */
+    lo = INFINITY;
+    hi = -INFINITY;
+#endif
+    for (int64_t k = 0; k < g; ++k) {
+        float v = wqo_bf16_to_f32(x[k]);
+        if (!isfinite(v)) flags |= WQO_FLAG_NONFINITE;
+        if (isnan(v)) continue;
+        if (v < lo) lo = v;
+        if (v > hi) hi = v;
+        float av = fabsf(v);
+        if (av > amax) amax = av;
+    }
+
+    /* scale in fp32, stored as fp16 */
+    float s32;
+    if (p->symmetric)
+        s32 = amax / (float)qmax;
+    else
+#if WQO_MUTANT == 3 /* mistake: divide by the level count, not the range */
+        s32 = (hi - lo) / (float)(qmax - qmin + 1);
+#else
+        s32 = (hi - lo) / (float)(qmax - qmin);
+#endif
+    uint16_t s16 = wqo_f32_to_f16(s32);
+    int z = 0;
+    if (s16 == 0x7c00u) { /* fp16 overflow: saturate */
+        s16 = 0x7bffu;
+        flags |= WQO_FLAG_RANGE;
+    }
+    if (s16 == 0x0000u) { /* all-zero or underflowing group */
+        s16 = 0x3c00u;  /* 1.0 */
+        z = 0;
+    } else if (!p->symmetric) {
+        float s = wqo_f16_to_f32(s16);
+        /* z = q_min - x_min/s, rounded (half to even) and clamped */
+#if WQO_MUTANT == 1 /* mistake: wrong sign of the zero point */
+        float zf = rintf((float)qmin + lo / s);
+#else
+        float zf = rintf((float)qmin - lo / s);
+#endif
+        z = clamp_to_int(zf, qmin, qmax);
+    }
+    float s = wqo_f16_to_f32(s16);
+
+    /* codes [P1 Affine]: q = clamp(round(x/s) + z, q_min, q_max) */
+    for (int64_t k = 0; k < g; ++k) {
+        float v = wqo_bf16_to_f32(x[k]);
+        if (isnan(v)) {
+            codes[k] = z; /* NaN is coded as zero */
+            continue;
+        }
+#if WQO_MUTANT == 2 /* mistake: round half away from zero */
+        float t = roundf(v / s);
+#else
+        float t = rintf(v / s);
+#endif
+        codes[k] = clamp_to_int(t + (float)z, qmin, qmax);
+    }
+    *s_out = s16;
+    if (z_out) *z_out = wqo_f32_to_f16((float)z);
+    return flags;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Row-parallel driver (pthreads over row ranges; the per-row code is the    */
+/* plain loop above).                                                        */
+/* ------------------------------------------------------------------------ */
+
+typedef void (*row_fn)(void* ctx, int64_t r0, int64_t r1, uint32_t* flags);
+
+typedef struct {
+    row_fn fn;
+    void* ctx;
+    int64_t r0, r1;
+    uint32_t flags;
+} row_job;
+
+static void* row_job_main(void* arg) {
+    row_job* j = (row_job*)arg;
+    j->flags = 0;
+    j->fn(j->ctx, j->r0, j->r1, &j->flags);
+    return NULL;
+}
+
+static uint32_t run_rows(row_fn fn, void* ctx, int64_t rows, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if ((int64_t)nthreads > rows) nthreads = rows > 0 ? (int)rows : 1;
+    row_job jobs[256];
+    pthread_t tids[256];
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t].fn = fn;
+        jobs[t].ctx = ctx;
+        jobs[t].r0 = rows * t / nthreads;
+        jobs[t].r1 = rows * (t + 1) / nthreads;
+    }
+    for (int t = 1; t < nthreads; ++t) pthread_create(&tids[t], NULL, row_job_main, &jobs[t]);
+    row_job_main(&jobs[0]);
+    uint32_t flags = jobs[0].flags;
+    for (int t = 1; t < nthreads; ++t) {
+        pthread_join(tids[t], NULL);
+        flags |= jobs[t].flags;
+    }
+    return flags;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantize                                                                  */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t* W;
+    int64_t d_in, g;
+    wqo_qparams p;
+    int32_t* codes;
+    uint16_t* scales;
+    uint16_t* zeros;
+} quant_ctx;
+
+static void quant_rows(void* vctx, int64_t r0, int64_t r1, uint32_t* flags) {
+    quant_ctx* c = (quant_ctx*)vctx;
+    int64_t ng = c->d_in / c->g;
+    for (int64_t r = r0; r < r1; ++r)
+        for (int64_t j = 0; j < ng; ++j) {
+            int64_t off = r * c->d_in + j * c->g;
+            *flags |= quantize_group(c->W + off, c->g, &c->p, c->codes + off,
+                                     c->scales + r * ng + j,
+                                     c->zeros ? c->zeros + r * ng + j : NULL);
+        }
+}
+
+/* W: bf16 bits [d_out][d_in]; codes: int32 [d_out][d_in];
+ * scales, zeros: fp16 bits [d_out][d_in/g] (zeros may be NULL when symmetric).
+ * Returns 0 on success, -1 on bad arguments; *flags gets WQO_FLAG_*. */
+int wqo_quantize(const uint16_t* W, int64_t d_out, int64_t d_in, int64_t g, int bits,
+                 int symmetric, int narrow, int32_t* codes, uint16_t* scales,
+                 uint16_t* zeros, uint32_t* flags, int nthreads) {
+    if (!W || !codes || !scales || d_out < 0 || d_in <= 0 || g <= 0 || d_in % g != 0)
+        return -1;
+    if (bits < 2 || bits > 8) return -1;
+    if (!symmetric && !zeros) return -1;
+    quant_ctx c = {W, d_in, g, {bits, symmetric, narrow}, codes, scales, symmetric ? NULL : zeros};
+    uint32_t f = run_rows(quant_rows, &c, d_out, nthreads);
+    if (flags) *flags = f;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Packing (4-bit only): 8 nibbles per uint32, low nibble first.             */
+/* ------------------------------------------------------------------------ */
+
+int wqo_pack4(const int32_t* codes, int64_t d_out, int64_t d_in, uint32_t* qweight) {
+    if (!codes || !qweight || d_in % 8 != 0) return -1;
+    for (int64_t r = 0; r < d_out; ++r)
+        for (int64_t c8 = 0; c8 < d_in / 8; ++c8) {
+            uint32_t w = 0;
+            for (int j = 0; j < 8; ++j) {
+                uint32_t nib = (uint32_t)codes[r * d_in + c8 * 8 + j] & 0xfu;
+#if WQO_MUTANT == 7 /* mistake: high nibble first */
+                w |= nib << (4 * (7 - j));
+#else
+                w |= nib << (4 * j);
+#endif
+            }
+            qweight[r * (d_in / 8) + c8] = w;
+        }
+    return 0;
+}
+
+/* Inverse of wqo_pack4: symmetric nibbles are read as 4-bit two's complement. */
+int wqo_unpack4(const uint32_t* qweight, int64_t d_out, int64_t d_in, int symmetric,
+                int32_t* codes) {
+    if (!codes || !qweight || d_in % 8 != 0) return -1;
+    for (int64_t r = 0; r < d_out; ++r)
+        for (int64_t c = 0; c < d_in; ++c) {
+            uint32_t w = qweight[r * (d_in / 8) + c / 8];
+            int32_t nib = (int32_t)((w >> (4 * (c % 8))) & 0xfu);
+            if (symmetric && nib >= 8) nib -= 16;
+            codes[r * d_in + c] = nib;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dequantize: x_hat = s (q - z), rounded once to bf16 [P1 Affine].          */
+/* ------------------------------------------------------------------------ */
+
+/* The product of an fp16 scale (11 significant bits) and an integer of at
+ * most 8 bits (|q - z| <= 255) has at most 19 significant bits and lies in
+ * the binary32 range, so it is exact in double and in float; the only
+ * rounding is the final one to bf16. */
+uint16_t wqo_dequant_one(uint16_t s16, int32_t q, int32_t z) {
+#if WQO_MUTANT == 6 /* mistake: zero point dropped */
+    z = 0;
+#endif
+    double prod = (double)wqo_f16_to_f32(s16) * (double)(q - z);
+    float pf = (float)prod; /* exact, see above */
+    return wqo_f32_to_bf16(pf);
+}
+
+typedef struct {
+    const int32_t* codes;
+    const uint16_t* scales;
+    const uint16_t* zeros;
+    int64_t d_in, g;
+    uint16_t* W_hat;
+} deq_ctx;
+
+static void deq_rows(void* vctx, int64_t r0, int64_t r1, uint32_t* flags) {
+    (void)flags;
+    deq_ctx* c = (deq_ctx*)vctx;
+    int64_t ng = c->d_in / c->g;
+    for (int64_t r = r0; r < r1; ++r)
+        for (int64_t k = 0; k < c->d_in; ++k) {
+            int64_t gi = r * ng + k / c->g;
+            int32_t z = c->zeros ? (int32_t)wqo_f16_to_f32(c->zeros[gi]) : 0;
+            c->W_hat[r * c->d_in + k] = wqo_dequant_one(c->scales[gi], c->codes[r * c->d_in + k], z);
+        }
+}
+
+/* codes int32 [d_out][d_in]; scales/zeros fp16 bits [d_out][d_in/g]
+ * (zeros NULL = symmetric); W_hat bf16 bits [d_out][d_in]. */
+int wqo_dequantize(const int32_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                   int64_t d_out, int64_t d_in, int64_t g, uint16_t* W_hat, int nthreads) {
+    if (!codes || !scales || !W_hat || g <= 0 || d_in % g != 0) return -1;
+    deq_ctx c = {codes, scales, zeros, d_in, g, W_hat};
+    run_rows(deq_rows, &c, d_out, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Linear: y[m,n] = sum_k W_hat[n,k] x[m,k] in fp64, plus the error scale    */
+/* A[m,n] = sum_k |W_hat[n,k] x[m,k]|.                                        */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t* X;
+    int64_t M;
+    const uint16_t* W_hat;
+    int64_t K;
+    double* Y;
+    double* A;
+    int64_t N;
+} lin_ctx;
+
+static void lin_rows(void* vctx, int64_t n0, int64_t n1, uint32_t* flags) {
+    (void)flags;
+    lin_ctx* c = (lin_ctx*)vctx;
+    for (int64_t n = n0; n < n1; ++n)
+        for (int64_t m = 0; m < c->M; ++m) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < c->K; ++k) {
+#if WQO_MUTANT == 5 /* mistake: transposed weight operand */
+                double t = (double)wqo_bf16_to_f32(c->W_hat[(k % c->N) * c->K + (n % c->K)]) *
+                           (double)wqo_bf16_to_f32(c->X[m * c->K + k]);
+#else
+                double t = (double)wqo_bf16_to_f32(c->W_hat[n * c->K + k]) *
+                           (double)wqo_bf16_to_f32(c->X[m * c->K + k]);
+#endif
+                acc += t;
+                aacc += fabs(t);
+            }
+            c->Y[m * c->N + n] = acc;
+            if (c->A) c->A[m * c->N + n] = aacc;
+        }
+}
+
+/* X bf16 bits [M][K]; W_hat bf16 bits [N][K]; Y, A fp64 [M][N] (A may be
+ * NULL).  Rows of W_hat are split across threads. */
+int wqo_linear(const uint16_t* X, int64_t M, const uint16_t* W_hat, int64_t N, int64_t K,
+               double* Y, double* A, int nthreads) {
+    if (!X || !W_hat || !Y || M < 0 || N < 0 || K < 0) return -1;
+    lin_ctx c = {X, M, W_hat, K, Y, A, N};
+    run_rows(lin_rows, &c, N, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Artifact bytes [P1 Memory arithmetic, Group scale overhead]:              */
+/*   payload = P * b / 8; one fp16 scale per group of g; one fp16 zero per   */
+/*   group when asymmetric.                                                  */
+/* ------------------------------------------------------------------------ */
+
+int wqo_artifact_bytes(int64_t params, int bits, int64_t g, int symmetric, double* payload,
+                       double* scale_bytes, double* zero_bytes) {
+    if (g <= 0 || bits <= 0) return -1;
+    *payload = (double)params * (double)bits / 8.0;
+    *scale_bytes = 2.0 * (double)params / (double)g;
+    *zero_bytes = symmetric ? 0.0 : 2.0 * (double)params / (double)g;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Array forms of the conversions (used by the pins to compare whole ranges  */
+/* of inputs against independent library conversions).                      */
+/* ------------------------------------------------------------------------ */
+
+void wqo_f32_to_f16_array(const float* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = wqo_f32_to_f16(x[i]);
+}
+
+void wqo_f32_to_bf16_array(const float* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = wqo_f32_to_bf16(x[i]);
+}
+
+void wqo_f16_to_f32_array(const uint16_t* h, int64_t n, float* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = wqo_f16_to_f32(h[i]);
+}

@@ -1,0 +1,51 @@
+"""Planted mistakes: each mutant of the oracle (one plausible error compiled
+in with -DWQO_MUTANT=k) must fail at least one pin, and the real oracle must
+pass the same pins.  This shows the pins constrain every step: statistics,
+scale, zero point, rounding, packing, dequantization and the linear layer."""
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+PINS = [
+    pins.test_zero_exactly_representable,
+    lambda: pins.test_rounding_error_bound(False),
+    pins.test_outlier20_asymmetric_and_clipping,
+    lambda: pins.test_round_trip_fixed_point(False),
+    lambda: pins.test_brute_force_argmin(-1.0, 1.5, False),
+    lambda: pins.test_brute_force_argmin(0.25, 7.0, False),
+    pins.test_pack_layout_low_nibble_first,
+    pins.test_dequant_exhaustive_against_library_rounding,
+    pins.test_linear_special_cases_and_matmul,
+]
+
+MUTANTS = {
+    1: "zero point sign",
+    2: "round half away from zero",
+    3: "scale divided by level count",
+    4: "range not widened to zero",
+    5: "transposed weight in linear",
+    6: "zero point dropped in dequant",
+    7: "high nibble first",
+}
+
+
+def _failures():
+    n = 0
+    for pin in PINS:
+        try:
+            pin()
+        except AssertionError:
+            n += 1
+    return n
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS), ids=lambda m: MUTANTS[m].replace(" ", "-"))
+def test_mutant_is_caught(mutant, tmp_path):
+    path = oracle.build_mutant(mutant, str(tmp_path))
+    with oracle.use_library(path):
+        assert _failures() >= 1, MUTANTS[mutant]
+
+
+def test_real_oracle_passes_the_same_pins():
+    assert _failures() == 0
