@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 hot path on B200 (one JSON line on stdout).
+
+Headline (the `value`): W4A16 decode GEMV GB/s on the Llama-7B attention
+projection workload -- W[4096, 4096] bf16 quantized group-128 asymmetric uint4,
+M = 1 bf16 activation.  One step = one decode sweep of 64 GEMV launches over 64
+distinct packed copies (557 MB of artifacts, > 4x the 126 MB L2, so every
+launch streams its weights from HBM), replayed from a CUDA graph.  Algorithmic
+bytes per launch: 0.5 B/weight packed codes + 4 B per group (fp16 scale+zero)
++ 2 B per activation in and output out = 8,929,280 B.
+
+The same line carries the other two metric items (quantize GB/s, GEMM
+TFLOP/s) and secondary decode shapes under "secondary", the roofline of the
+dominant kernel, an end-to-end number through the C ABI with host buffers,
+clocks sampled during the timed regions, and the CPU-oracle baseline.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With N > 1 (torchrun) every rank runs an independent replica (the path does
+not shard: "replicas only"); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 GEMV GB/s & %HBM roofline (4096², g128, M=1); quantize GB/s; GEMM TFLOP/s"
+NCOPY = 64
+D = 4096
+G128 = 128
+
+
+def gemv_bytes(N: int, K: int, M: int, symmetric: bool, g: int = 128) -> int:
+    per_group = 2 if symmetric else 4
+    return N * K // 2 + (N * K // g) * per_group + 2 * M * (K + N)
+
+
+def quant_bytes(N: int, K: int, symmetric: bool, g: int = 128) -> int:
+    per_group = 2 if symmetric else 4
+    return N * K * 2 + N * K // 2 + (N * K // g) * per_group
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (replicas only: a barrier and a max of timings)
+# --------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed regions
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="wq_clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if self.proc is None:
+            return out
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return out
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, flags in rows:
+            for n, v in zip(names, flags):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        out["sm_mhz"] = statistics.median(r[0] for r in rows)
+        out["sm_max_mhz"] = max(r[1] for r in rows)
+        out["reasons"] = sorted(reasons)
+        out["samples"] = len(rows)
+        return out
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def timed_graph(graph: torch.cuda.CUDAGraph, steps: int, warmup: int, dist: Dist):
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        graph.replay()
+    e.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    return s.elapsed_time(e) / 1e3  # seconds
+
+
+def capture(fn) -> torch.cuda.CUDAGraph:
+    fn()  # eager warm-up (first-call set-up happens outside the capture)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def replicate(p, n):
+    from w4a16_bit_gemm_b200 import binding as b
+    return [b.PackedLinear(p.qweight.clone(), p.scales.clone(), None if p.zeros is None else p.zeros.clone(),
+                           p.d_out, p.d_in, p.group_size, p.symmetric) for _ in range(n)]
+
+
+def gemv_sweep(b, packs, X, Y):
+    def fn():
+        for i, p in enumerate(packs):
+            b.linear_w4a16(X[i], p, out=Y[i])
+    return fn
+
+
+def bench_gemv_shape(b, syn, wl, ci, M, copies, steps, warmup, dist):
+    c = wl.cases[ci]
+    W = syn.case_weight(wl, ci, "cuda")
+    p0 = b.quantize_rtn(W, c.group_size, c.symmetric)
+    del W
+    packs = replicate(p0, copies)
+    X = [syn.case_activations(wl, ci, M, "cuda") for _ in range(1)] * copies
+    Y = [torch.empty(M, c.d_out, dtype=torch.bfloat16, device="cuda") for _ in range(copies)]
+    g = capture(gemv_sweep(b, packs, X, Y))
+    t = dist.max(timed_graph(g, steps, warmup, dist))
+    per_launch = t / (steps * copies)
+    nbytes = gemv_bytes(c.d_out, c.d_in, M, c.symmetric, c.group_size)
+    del g, packs, Y
+    torch.cuda.empty_cache()
+    return {"shape": f"{c.d_out}x{c.d_in}", "M": M, "symmetric": c.symmetric, "us_per_launch": per_launch * 1e6,
+            "GBps": nbytes / per_launch / 1e9, "bytes_per_launch": nbytes}
+
+
+def run_ours(args, dist: Dist):
+    from w4a16_bit_gemm_b200 import binding as b
+    from w4a16_bit_gemm_b200 import synthetic as syn
+
+    hbm, tf_burst, tf_sust, peak_src = load_peaks()
+    dev = torch.cuda.current_device()
+    sampler = ClockSampler(dev)
+
+    # ---------------- headline: cfg2 GEMV M=1 decode sweep ----------------
+    wl = syn.ATTN
+    c = wl.cases[0]
+    W = syn.case_weight(wl, 0, "cuda")
+    p0 = b.quantize_rtn(W, G128, False)
+    packs = replicate(p0, NCOPY)
+    X_all = syn.activations(NCOPY, D, wl.seed, 77, "cuda", channel_outlier_frac=0.001)
+    Y_all = torch.empty(NCOPY, D, dtype=torch.bfloat16, device="cuda")
+    Xv = [X_all[i:i + 1] for i in range(NCOPY)]
+    Yv = [Y_all[i:i + 1] for i in range(NCOPY)]
+    graph = capture(gemv_sweep(b, packs, Xv, Yv))
+    st, flags = b.device_error()
+    if st != b.WQ_OK:
+        raise RuntimeError(f"device status after warm-up: {st} flags {flags}")
+
+    sampler.start()
+    t_head = dist.max(timed_graph(graph, args.steps, args.warmup, dist))
+    per_launch = t_head / (args.steps * NCOPY)
+    bytes_launch = gemv_bytes(D, D, 1, False)
+    value = bytes_launch * NCOPY * args.steps * dist.world / t_head / 1e9
+    achieved = bytes_launch / per_launch / 1e9
+
+    # ---------------- end to end through the C ABI with host buffers ----------------
+    X_host = X_all.cpu().pin_memory()
+    Y_host = torch.empty_like(Y_all, device="cpu").pin_memory()
+    stream = torch.cuda.current_stream()
+    e2e_steps = max(10, min(args.steps, 500))
+    for _ in range(3):
+        X_all.copy_(X_host, non_blocking=True)
+        graph.replay()
+        Y_host.copy_(Y_all, non_blocking=True)
+        stream.synchronize()
+    dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        X_all.copy_(X_host, non_blocking=True)
+        graph.replay()
+        Y_host.copy_(Y_all, non_blocking=True)
+        stream.synchronize()
+    t_e2e = dist.max(time.perf_counter() - t0)
+    dist.barrier()
+    e2e_value = bytes_launch * NCOPY * e2e_steps * dist.world / t_e2e / 1e9
+    del graph, packs
+
+    # ---------------- secondary: quantize GB/s, dequant GB/s ----------------
+    secondary = {}
+    QC = 16
+    Ws = [W] + [W.clone() for _ in range(QC - 1)]
+    qpacks = replicate(p0, QC)
+
+    def qfn():
+        for i in range(QC):
+            b.quantize_rtn(Ws[i], G128, False, out=qpacks[i])
+    gq = capture(qfn)
+    qsteps = max(5, args.steps // 20)
+    tq = dist.max(timed_graph(gq, qsteps, 3, dist)) / (qsteps * QC)
+    qb = quant_bytes(D, D, False)
+    secondary["quantize"] = {"shape": "4096x4096", "GBps": qb / tq / 1e9, "us_per_launch": tq * 1e6,
+                             "bytes_per_launch": qb, "frac_of_measured_hbm": qb / tq / 1e9 / hbm}
+    What = [torch.empty(D, D, dtype=torch.bfloat16, device="cuda") for _ in range(QC)]
+
+    def dfn():
+        for i in range(QC):
+            b.dequantize(qpacks[i], out=What[i])
+    gd = capture(dfn)
+    td = dist.max(timed_graph(gd, qsteps, 3, dist)) / (qsteps * QC)
+    secondary["dequantize"] = {"shape": "4096x4096", "GBps": qb / td / 1e9, "us_per_launch": td * 1e6,
+                               "frac_of_measured_hbm": qb / td / 1e9 / hbm}
+    del gq, gd, Ws, qpacks, What, W
+    torch.cuda.empty_cache()
+
+    # ---------------- secondary decode shapes ----------------
+    ssteps = max(5, args.steps // 10)
+    secondary["gemv"] = []
+    for (wlx, ci, M) in ((syn.ATTN, 0, 8), (syn.MLP, 0, 1), (syn.MLP, 0, 16), (syn.MLP, 2, 1), (syn.MLP, 2, 4)):
+        r = bench_gemv_shape(b, syn, wlx, ci, M, 24, ssteps, 3, dist)
+        r["frac_of_measured_hbm"] = r["GBps"] / hbm
+        secondary["gemv"].append(r)
+
+    # ---------------- GEMM TFLOP/s (config 4) ----------------
+    secondary["gemm"] = []
+    for (ci, M) in ((0, 512), (0, 2048), (1, 8192)):
+        cc = syn.PREFILL.cases[ci]
+        Wg = syn.case_weight(syn.PREFILL, ci, "cuda")
+        pg = b.quantize_rtn(Wg, G128, False)
+        del Wg
+        Xg = syn.case_activations(syn.PREFILL, ci, M, "cuda")
+        Yg = torch.empty(M, cc.d_out, dtype=torch.bfloat16, device="cuda")
+        gg = capture(lambda: b.linear_w4a16(Xg, pg, out=Yg))
+        gsteps = max(3, min(50, args.steps // 40))
+        tg = dist.max(timed_graph(gg, gsteps, 2, dist)) / gsteps
+        flops = 2.0 * M * cc.d_out * cc.d_in
+        tfl = flops / tg / 1e12
+        secondary["gemm"].append({"M": M, "N": cc.d_out, "K": cc.d_in, "ms_per_launch": tg * 1e3, "TFLOPs": tfl,
+                                  "frac_of_measured_bf16_burst": tfl / tf_burst,
+                                  "frac_of_measured_bf16_sustained": tfl / tf_sust})
+        del gg, pg, Xg, Yg
+        torch.cuda.empty_cache()
+    clocks = sampler.stop()
+    st, flags = b.device_error()
+    if st != b.WQ_OK:
+        raise RuntimeError(f"device status after the bench: {st} flags {flags}")
+
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "gemv_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                traffic = json.load(f).get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_head / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 activations x uint4 weights, fp32 accumulate",
+        "data": "synthetic (seeded N(0,0.02) weights with 0.1% column outliers x20; N(0,1) activations with 0.1% channels x50)",
+        "config": {"workload": "llama7b-attn-proj W[4096,4096] g128 asym uint4, W4A16 GEMV M=1",
+                   "step": f"{NCOPY} GEMV launches over {NCOPY} distinct packed copies (CUDA graph)",
+                   "l2": f"inputs larger than L2: {NCOPY} artifact copies = {NCOPY * p0.nbytes() / 1e6:.0f} MB",
+                   "parallelism": f"replicas x{dist.world}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic, "peak_source": f"{peak_src} hbm_gbs"},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": NCOPY * D * 2,
+                "d2h_bytes_per_step": NCOPY * D * 2},
+        "gpu_launches": args.steps * NCOPY,
+        "clocks": clocks,
+        "secondary": secondary,
+    }
+    return out
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# --------------------------------------------------------------------------
+
+def oracle_gemv_sample(n_launch: int):
+    """The oracle as it stands on the same workload: for each launch of the
+    sample, unpack the artifact, dequantize and run the fp64 linear layer."""
+    import oracle
+    from w4a16_bit_gemm_b200 import synthetic as syn
+    W = syn.case_weight(syn.ATTN, 0, "cpu")
+    Wb = W.view(torch.int16).numpy().view(np.uint16)
+    q, s, z, _, _ = oracle.quantize_pack4(Wb, 128, False)
+    X = syn.activations(1, D, syn.ATTN.seed, 77, "cpu", channel_outlier_frac=0.001)
+    Xb = X.view(torch.int16).numpy().view(np.uint16)
+    nthreads = oracle.default_threads()
+    t0 = time.perf_counter()
+    for _ in range(n_launch):
+        codes = oracle.unpack4(q, D, False)
+        W_hat = oracle.dequantize(codes, s, z, 128, nthreads)
+        oracle.linear(Xb, W_hat, nthreads)
+    dt = time.perf_counter() - t0
+    return gemv_bytes(D, D, 1, False) * n_launch / dt / 1e9, nthreads, dt
+
+
+def calibrated_sample(target_s: float = 12.0):
+    v, n, dt = oracle_gemv_sample(1)
+    per = dt
+    n_launch = max(1, min(200, int(target_s / max(per, 1e-3))))
+    v, n, dt = oracle_gemv_sample(n_launch)
+    return v, n, dt, n_launch
+
+
+def run_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return None
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_gemv_sample(1)
+    v, n, dt = oracle_gemv_sample(max(1, args.steps // 200))
+    n_launch = max(1, args.steps // 200)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": v,
+        "unit": "GB/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp64 accumulate over bf16 dequantized weights (CPU oracle)",
+        "data": "synthetic (same seeded workload)",
+        "config": {"workload": "llama7b-attn-proj W[4096,4096] g128 asym uint4, W4A16 GEMV M=1",
+                   "step": f"{n_launch} oracle GEMV(s): unpack + dequantize + fp64 linear"},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": n, "kind": "oracle",
+                         "sample": f"{n_launch} GEMV launch(es) of the 4096x4096 M=1 workload"},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    dist = Dist()
+    try:
+        if args.impl == "reference":
+            out = run_reference(args, dist)
+        else:
+            out = run_ours(args, dist)
+            if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+                v, n, dt, nl = calibrated_sample()
+                out["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": n, "kind": "oracle",
+                                       "sample": f"{nl} GEMV launch(es) of the 4096x4096 M=1 workload "
+                                                 f"(unpack + dequantize + fp64 linear), {dt:.1f} s"}
+        if out is not None and dist.rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

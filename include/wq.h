@@ -1,0 +1,186 @@
+/*
+ * wq.h -- C ABI of libwq: group-wise RTN 4-bit weight quantization,
+ * dequantization and W4A16 linear layers on NVIDIA B200 (sm_100a).
+ *
+ * The operations are the ones defined on
+ *   "LLM Quantization: GPTQ, AWQ, SmoothQuant, FP8, KV Cache (7/10)"
+ *   (blog.ruahverce.com), sections "Affine Quantization" (q = clamp(round(x/s)
+ *   + z, q_min, q_max); x_hat = s (q - z)), "Symmetric and Asymmetric",
+ *   "Per-group" (group_size = 128, one scale per 128 weights), and "Fused
+ *   low-bit kernel" (packed INT4 weights -> fused load/dequant/matmul ->
+ *   higher-precision accumulation),
+ * with the code ranges of "Quantization Algorithms" (V10 study notes,
+ * brianyu43.github.io), section 1.8 (INT4 signed [-8,7], asymmetric unsigned
+ * [0,15]).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All array arguments are DEVICE pointers owned by the caller.  The library
+ *   never frees or retains them.  The library owns only one device status
+ *   word per device (a static device variable; no entry point allocates
+ *   device memory).  The first call on a device looks up that word's address
+ *   and should not be made inside a stream capture.
+ * - Matrices are dense row-major.  bf16 and fp16 values are passed as their
+ *   16-bit storage (void*).
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *   call is asynchronous on that stream: it returns once the work is
+ *   enqueued.  Only wq_get_device_error synchronizes.
+ * - Argument errors are detected on the host and returned synchronously with
+ *   nothing launched.  A failed launch returns WQ_ERR_CUDA.  Conditions found
+ *   on the device (non-finite input, fp16 scale overflow, a pipeline wait that
+ *   gave up) set bits in the device status word, read with
+ *   wq_get_device_error.  No entry point traps, asserts or throws.
+ *
+ * Packed layout v1 (WQ_LAYOUT_V1)
+ * -------------------------------
+ * - qweight: uint32 [d_out][d_in/8].  Nibble j (bits 4j..4j+3, low nibble
+ *   first) of word c of row r holds the code of column 8c+j.  Asymmetric codes
+ *   are unsigned 0..15; symmetric codes are 4-bit two's complement -8..7.
+ * - scales: fp16 [d_out][d_in/group_size] (row-major, group index fastest).
+ * - zeros:  fp16 [d_out][d_in/group_size] holding integers 0..15 (asymmetric
+ *   only; NULL for symmetric, where z = 0).
+ * - The group axis is the input dimension d_in: group j of row r covers
+ *   columns [j*group_size, (j+1)*group_size).
+ *
+ * Numerics
+ * --------
+ * - Asymmetric: x_min' = min(0, min x), x_max' = max(0, max x);
+ *   s = fp16_rn(fp32(x_max' - x_min') / 15); z = clamp(rint(-x_min'/s), 0, 15).
+ *   Symmetric: s = fp16_rn(max|x| / 7), z = 0.  A zero fp16 scale becomes
+ *   s = 1, z = 0; an fp16 overflow saturates s to 65504 (WQ_DEVFLAG_RANGE).
+ * - Codes: q = clamp(rint(fp32(x) / s) + z, q_min, q_max) with an IEEE fp32
+ *   division by the stored fp16 scale and round-half-to-even.  NaN inputs are
+ *   skipped by the statistics and coded as z (WQ_DEVFLAG_NONFINITE).
+ * - Dequantization: x_hat = bf16_rn(s * (q - z)), one rounding of the exact
+ *   product.
+ * - Linear: y[m,n] = sum_k x_hat[n,k] * x[m,k] with bf16 x_hat exactly as
+ *   above and fp32 accumulation ("dequantize, then multiply in floating
+ *   point", one rounding of the dequantized weight).
+ */
+#ifndef WQ_H_
+#define WQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WQ_ABI_VERSION 1
+#define WQ_LAYOUT_V1 1
+
+typedef enum {
+    WQ_OK = 0,
+    WQ_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or group size */
+    WQ_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+    WQ_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
+    WQ_ERR_NONFINITE = 4,   /* returned by wq_get_device_error: NaN/Inf input seen */
+    WQ_ERR_TIMEOUT = 5,     /* returned by wq_get_device_error: a device wait gave up */
+    WQ_ERR_RANGE = 6        /* returned by wq_get_device_error: fp16 scale saturated */
+} wq_status;
+
+/* Bits of the device status word. */
+#define WQ_DEVFLAG_NONFINITE 0x1u
+#define WQ_DEVFLAG_RANGE 0x2u
+#define WQ_DEVFLAG_TIMEOUT 0x4u
+
+/* Output element types of wq_linear_w4a16. */
+#define WQ_OUT_BF16 0
+#define WQ_OUT_FP32 1
+
+/* ABI version of the loaded library (WQ_ABI_VERSION). */
+int32_t wq_abi_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* wq_status_string(wq_status status);
+
+/*
+ * wq_quantize_rtn -- group-wise round-to-nearest affine quantization to packed
+ * 4-bit codes ("Affine Quantization", "Symmetric and Asymmetric",
+ * "Per-group" sections of the first page cited above).
+ *
+ *   W_bf16      [d_out][d_in] bf16, input.  16-byte aligned.
+ *   d_out       rows (output channels), >= 1.
+ *   d_in        columns (input channels), >= 1, multiple of group_size.
+ *   group_size  32, 64, 128, 256, or a multiple of 256; divides d_in.
+ *   symmetric   0: uint4 [0,15] with zeros; 1: int4 [-8,7], zeros_fp16 NULL.
+ *   qweight     [d_out][d_in/8] uint32 output (layout v1).  16-byte aligned.
+ *   scales_fp16 [d_out][d_in/group_size] fp16 output.  2-byte aligned.
+ *   zeros_fp16  [d_out][d_in/group_size] fp16 output (asymmetric), else NULL.
+ *
+ * Errors: WQ_ERR_INVALID_ARG for null/misaligned pointers, non-positive sizes,
+ * a group size that does not divide d_in or is not supported, zeros_fp16 NULL
+ * with symmetric == 0, or zeros_fp16 non-NULL with symmetric == 1.
+ * Device flags: WQ_DEVFLAG_NONFINITE, WQ_DEVFLAG_RANGE.
+ */
+wq_status wq_quantize_rtn(const void* W_bf16, int64_t d_out, int64_t d_in, int32_t group_size,
+                          int32_t symmetric, uint32_t* qweight, void* scales_fp16,
+                          void* zeros_fp16, void* stream);
+
+/*
+ * wq_dequantize -- x_hat = bf16_rn(s (q - z)) for every weight ("Affine
+ * Quantization"; the "full dequantize then matmul" path B of the "Fused
+ * low-bit kernel" section).  Arguments as in wq_quantize_rtn, with the packed
+ * artifact as input and
+ *   W_hat_bf16  [d_out][d_in] bf16 output.  16-byte aligned.
+ * zeros_fp16 must hold integers 0..15 (other values give unspecified but
+ * memory-safe results).
+ */
+wq_status wq_dequantize(const uint32_t* qweight, const void* scales_fp16, const void* zeros_fp16,
+                        int64_t d_out, int64_t d_in, int32_t group_size, int32_t symmetric,
+                        void* W_hat_bf16, void* stream);
+
+/*
+ * wq_linear_w4a16 -- Y[M][d_out] = X[M][d_in] . x_hat^T, the W4A16 linear
+ * layer consuming the packed artifact (path A, "Fused low-bit kernel":
+ * packed INT4 weights -> fused load/dequant/matmul -> fp32 accumulation).
+ *
+ *   X_bf16      [M][d_in] bf16 activations, input.  16-byte aligned.
+ *   M           tokens, >= 1.  M <= 16 runs the decode GEMV kernel; larger M
+ *               runs the tcgen05 tensor-core GEMM kernel.
+ *   qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric:
+ *               the packed artifact, as produced by wq_quantize_rtn.
+ *   Y           [M][d_out] output, bf16 (y_dtype = WQ_OUT_BF16) or fp32
+ *               (WQ_OUT_FP32).  16-byte aligned.
+ *   workspace, workspace_bytes
+ *               scratch owned by the caller, at least
+ *               wq_linear_workspace_bytes(M, d_out, d_in) bytes (may be NULL
+ *               when that is 0).  Its contents on entry do not matter.
+ *
+ * Errors: WQ_ERR_INVALID_ARG as for wq_quantize_rtn, plus M < 1, a bad
+ * y_dtype or a workspace that is too small.
+ * Device flags: WQ_DEVFLAG_TIMEOUT if a pipeline wait inside the kernel gave
+ * up (the output is then incomplete).
+ */
+wq_status wq_linear_w4a16(const void* X_bf16, int64_t M, const uint32_t* qweight,
+                          const void* scales_fp16, const void* zeros_fp16, int64_t d_out,
+                          int64_t d_in, int32_t group_size, int32_t symmetric, void* Y,
+                          int32_t y_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Scratch bytes wq_linear_w4a16 needs for this shape (0 when none). */
+size_t wq_linear_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in);
+
+/*
+ * wq_get_device_error -- synchronize `stream`, read and clear the device
+ * status word of the current device.  *flags receives the WQ_DEVFLAG_* bits
+ * (may be NULL).  Returns WQ_OK when no bit was set, otherwise the status of
+ * the most severe bit (TIMEOUT, then NONFINITE, then RANGE), or WQ_ERR_CUDA.
+ */
+wq_status wq_get_device_error(uint32_t* flags, void* stream);
+
+/*
+ * wq_selftest_bounded_wait -- failure-detection self test (the pages have no
+ * counterpart; it exercises the bounded waits every pipeline kernel uses).
+ * Launches one CTA that waits on an mbarrier nothing arrives on, with a limit
+ * of `limit_us` microseconds (1 .. 1,000,000).  The wait gives up, sets
+ * WQ_DEVFLAG_TIMEOUT and the kernel exits normally; a following
+ * wq_get_device_error returns WQ_ERR_TIMEOUT and the context stays usable.
+ */
+wq_status wq_selftest_bounded_wait(uint32_t limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H_ */

@@ -1,0 +1,87 @@
+"""C-ABI library: loads, exports every symbol include/wq.h declares, and the
+host-side validation rejects bad arguments before any CUDA call (runs without
+a GPU: no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4a16_bit_gemm_b200 import build
+    build.build()
+    from w4a16_bit_gemm_b200 import binding
+    return binding.lib
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(wq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("wq_quantize_rtn", "wq_dequantize", "wq_linear_w4a16", "wq_linear_workspace_bytes",
+              "wq_get_device_error", "wq_status_string", "wq_abi_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.wq_abi_version() == 1
+    for code, name in [(0, b"WQ_OK"), (1, b"WQ_ERR_INVALID_ARG"), (3, b"WQ_ERR_CUDA"), (5, b"WQ_ERR_TIMEOUT")]:
+        assert lib.wq_status_string(code) == name
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("case", [
+    dict(W=None),
+    dict(W=FAKE + 2),                        # misaligned input
+    dict(q=FAKE + 4),                        # misaligned qweight
+    dict(d_out=0),
+    dict(d_in=0),
+    dict(g=100),                             # not a supported group size
+    dict(d_in=1000, g=128),                  # group does not divide d_in
+    dict(g=384, d_in=768),                   # > 256 and not a multiple of 256
+    dict(zeros=None),                        # asymmetric without zeros
+    dict(sym=1),                             # symmetric with zeros
+    dict(sym=2),
+])
+def test_quantize_rejects(lib, case):
+    a = dict(W=FAKE, d_out=4, d_in=256, g=128, sym=0, q=FAKE, s=FAKE, zeros=FAKE)
+    a.update(case)
+    st = lib.wq_quantize_rtn(a["W"], a["d_out"], a["d_in"], a["g"], a["sym"], a["q"], a["s"], a["zeros"], None)
+    assert st == 1
+
+
+@pytest.mark.parametrize("case", [
+    dict(X=None), dict(Y=None), dict(X=FAKE + 8), dict(M=0), dict(ydt=2), dict(g=48), dict(sym=1),
+])
+def test_linear_rejects(lib, case):
+    a = dict(X=FAKE, M=1, q=FAKE, s=FAKE, z=FAKE, N=64, K=256, g=128, sym=0, Y=FAKE, ydt=0)
+    a.update(case)
+    st = lib.wq_linear_w4a16(a["X"], a["M"], a["q"], a["s"], a["z"], a["N"], a["K"], a["g"], a["sym"], a["Y"],
+                             a["ydt"], None, 0, None)
+    assert st == 1
+
+
+def test_dequantize_rejects(lib):
+    assert lib.wq_dequantize(FAKE, FAKE, FAKE, 4, 256, 128, 0, None, None) == 1
+    assert lib.wq_dequantize(None, FAKE, FAKE, 4, 256, 128, 0, FAKE, None) == 1
+    assert lib.wq_dequantize(FAKE, FAKE, None, 4, 256, 128, 0, FAKE, None) == 1
+
+
+def test_workspace_query(lib):
+    assert lib.wq_linear_workspace_bytes(1, 4096, 4096) >= 0

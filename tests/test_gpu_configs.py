@@ -1,0 +1,118 @@
+"""The five seeded workloads at full size, on the GPU, against the oracle.
+
+Configs 1-3 are checked completely (every code, scale, zero and output);
+configs 4 and 5 on sampled rows / outputs the oracle computes one by one,
+in the same launch configuration the benchmark times.  Packed artifacts are
+bit-exact; linear outputs satisfy |y - y_ref| <= 1e-3 * sum|w_hat x| + 1e-6."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests._util import bits16, bits32, linear_tolerance_ok
+from w4a16_bit_gemm_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+
+def _b():
+    from w4a16_bit_gemm_b200 import binding
+    return binding
+
+
+def check_full_case(wl, ci, Ms, device_gen="cpu"):
+    b = _b()
+    c = wl.cases[ci]
+    W = syn.case_weight(wl, ci, device_gen)
+    Wb = bits16(W)
+    b.device_error()
+    p = b.quantize_rtn(W.cuda(), c.group_size, c.symmetric)
+    st, flags = b.device_error()
+    oq, os_, oz, of, codes = oracle.quantize_pack4(Wb, c.group_size, c.symmetric)
+    assert np.array_equal(bits32(p.qweight), oq)
+    assert np.array_equal(bits16(p.scales), os_)
+    if not c.symmetric:
+        assert np.array_equal(bits16(p.zeros), oz)
+    assert flags == of
+    W_hat_ref = oracle.dequantize(codes, os_, oz, c.group_size)
+    assert np.array_equal(bits16(b.dequantize(p)), W_hat_ref)
+    for M in Ms:
+        X = syn.case_activations(wl, ci, M, device_gen)
+        Y = b.linear_w4a16(X.cuda(), p)
+        y_ref, A = oracle.linear(bits16(X), W_hat_ref)
+        ok, ratio = linear_tolerance_ok(Y.float().cpu().numpy(), y_ref, A)
+        assert ok, (c.name, M, ratio)
+
+
+def test_config1_tiny():
+    check_full_case(syn.TINY, 0, (1,))
+
+
+def test_config2_attention_projection():
+    check_full_case(syn.ATTN, 0, (1, 8))
+
+
+@pytest.mark.parametrize("ci", [0, 1, 2], ids=["gate", "up", "down"])
+def test_config3_mlp(ci):
+    check_full_case(syn.MLP, ci, (1, 4, 16))
+
+
+@pytest.mark.parametrize("ci", [0, 1], ids=["8192x8192", "28672x8192"])
+def test_config4_prefill_sampled(ci):
+    b = _b()
+    wl = syn.PREFILL
+    c = wl.cases[ci]
+    rng = np.random.default_rng(40 + ci)
+    W = syn.case_weight(wl, ci, "cuda")
+    p = b.quantize_rtn(W, c.group_size, c.symmetric)
+    cols = np.sort(np.r_[rng.choice(c.d_out, 96, replace=False), [0, 255, 256, c.d_out - 1]])
+    Wb_s = bits16(W[torch.from_numpy(cols).cuda()])
+    oq, os_, oz, _, codes = oracle.quantize_pack4(Wb_s, c.group_size, c.symmetric)
+    idx = torch.from_numpy(cols).cuda()
+    assert np.array_equal(bits32(p.qweight[idx]), oq)
+    assert np.array_equal(bits16(p.scales[idx]), os_)
+    assert np.array_equal(bits16(p.zeros[idx]), oz)
+    W_hat_s = oracle.dequantize(codes, os_, oz, c.group_size)
+    del W
+    for M in c.Ms:
+        X = syn.case_activations(wl, ci, M, "cuda")
+        Y = b.linear_w4a16(X, p)
+        rows = np.sort(np.r_[rng.choice(M, 48, replace=False), [0, M - 1]])
+        ridx = torch.from_numpy(rows).cuda()
+        y = Y[ridx][:, idx].float().cpu().numpy()
+        y_ref, A = oracle.linear(bits16(X[ridx]), W_hat_s)
+        ok, ratio = linear_tolerance_ok(y, y_ref, A)
+        assert ok, (c.name, M, ratio)
+        st, flags = b.device_error()
+        assert st == b.WQ_OK
+        del X, Y
+
+
+def test_config5_whole_model_sampled():
+    """Quantize all 160 tensors of the 32-layer decoder (artifact bytes equal
+    P*4/8 + fp16 scale and zero per group), then the per-layer M=1 GEMV sweep;
+    each tensor checked on sampled rows."""
+    b = _b()
+    wl = syn.WHOLE_MODEL
+    rng = np.random.default_rng(50)
+    total_bytes = 0
+    for ci, c in enumerate(wl.cases):
+        W = syn.case_weight(wl, ci, "cuda")
+        p = b.quantize_rtn(W, c.group_size, c.symmetric)
+        total_bytes += p.nbytes()
+        rows = np.sort(np.r_[rng.choice(c.d_out, 6, replace=False), [c.d_out - 1]])
+        ridx = torch.from_numpy(rows).cuda()
+        oq, os_, oz, _, codes = oracle.quantize_pack4(bits16(W[ridx]), c.group_size, c.symmetric)
+        assert np.array_equal(bits32(p.qweight[ridx]), oq), c.name
+        assert np.array_equal(bits16(p.scales[ridx]), os_), c.name
+        assert np.array_equal(bits16(p.zeros[ridx]), oz), c.name
+        X = syn.case_activations(wl, ci, 1, "cuda")
+        Y = b.linear_w4a16(X, p)
+        y_ref, A = oracle.linear(bits16(X), oracle.dequantize(codes, os_, oz, c.group_size))
+        ok, ratio = linear_tolerance_ok(Y[:, ridx].float().cpu().numpy(), y_ref, A)
+        assert ok, (c.name, ratio)
+        del W, p, X, Y
+    payload, sb, zb = oracle.artifact_bytes(syn.total_params(wl), 4, 128, False)
+    assert total_bytes == payload + sb + zb == 3_440_377_856
+    st, flags = b.device_error()
+    assert st == b.WQ_OK

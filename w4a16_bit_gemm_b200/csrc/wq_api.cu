@@ -1,0 +1,245 @@
+// wq_api.cu -- the extern "C" boundary of libwq (declared in include/wq.h).
+//
+// Host-side argument validation, the per-device status word, tensor-map
+// encoding through the driver entry point, and dispatch to the kernels.
+// No entry point allocates device memory: the status word is a static device
+// variable and every other buffer belongs to the caller.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/wq.h"
+#include "wq_kernels.h"
+
+namespace wq {
+
+// Device status word (WQ_DEVFLAG_* bits), one per device that loads the library.
+__device__ uint32_t g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+uint32_t* g_status_ptr[kMaxDevices];
+int g_num_sms[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct DeviceState {
+    int dev;
+    uint32_t* status;
+    int num_sms;
+};
+
+// Per-device set-up on first use: address of the status word, SM count.
+// Must not run inside a stream capture (it may load the module).
+wq_status device_state(DeviceState* st) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return WQ_ERR_CUDA;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WQ_ERR_CUDA;
+        g_num_sms[dev] = sms;
+        g_status_ptr[dev] = static_cast<uint32_t*>(p);
+    }
+    st->dev = dev;
+    st->status = g_status_ptr[dev];
+    st->num_sms = g_num_sms[dev];
+    return WQ_OK;
+}
+
+bool group_size_ok(int64_t d_in, int32_t g) {
+    if (g <= 0 || d_in % g != 0) return false;
+    if (g == 32 || g == 64 || g == 128 || g == 256) return true;
+    return g % 256 == 0;
+}
+
+wq_status check_artifact(const void* qweight, const void* scales, const void* zeros, int64_t d_out, int64_t d_in,
+                         int32_t g, int32_t symmetric) {
+    if (!qweight || !scales) return WQ_ERR_INVALID_ARG;
+    if (d_out < 1 || d_in < 1 || d_out > (1ll << 31) - 1 || d_in > (1ll << 31) - 1) return WQ_ERR_INVALID_ARG;
+    if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+    if (!group_size_ok(d_in, g)) return WQ_ERR_INVALID_ARG;
+    if (symmetric == 0 && !zeros) return WQ_ERR_INVALID_ARG;
+    if (symmetric == 1 && zeros) return WQ_ERR_INVALID_ARG;
+    if (!aligned(qweight, 16) || !aligned(scales, 2) || (zeros && !aligned(zeros, 2))) return WQ_ERR_INVALID_ARG;
+    return WQ_OK;
+}
+
+bool pdl_enabled() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("WQ_DISABLE_PDL");
+        v = (e && e[0] == '1') ? 0 : 1;
+    }
+    return v == 1;
+}
+
+}  // namespace
+
+CUresult encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                              uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                              CUtensorMapSwizzle swizzle) {
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return CUDA_ERROR_NOT_FOUND;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+    }
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_stride_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+}  // namespace wq
+
+using namespace wq;
+
+extern "C" {
+
+int32_t wq_abi_version(void) { return WQ_ABI_VERSION; }
+
+const char* wq_status_string(wq_status s) {
+    switch (s) {
+        case WQ_OK: return "WQ_OK";
+        case WQ_ERR_INVALID_ARG: return "WQ_ERR_INVALID_ARG";
+        case WQ_ERR_UNSUPPORTED: return "WQ_ERR_UNSUPPORTED";
+        case WQ_ERR_CUDA: return "WQ_ERR_CUDA";
+        case WQ_ERR_NONFINITE: return "WQ_ERR_NONFINITE";
+        case WQ_ERR_TIMEOUT: return "WQ_ERR_TIMEOUT";
+        case WQ_ERR_RANGE: return "WQ_ERR_RANGE";
+    }
+    return "WQ_ERR_UNKNOWN";
+}
+
+wq_status wq_quantize_rtn(const void* W_bf16, int64_t d_out, int64_t d_in, int32_t group_size, int32_t symmetric,
+                          uint32_t* qweight, void* scales_fp16, void* zeros_fp16, void* stream) {
+    if (!W_bf16 || !aligned(W_bf16, 16)) return WQ_ERR_INVALID_ARG;
+    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
+    if (v != WQ_OK) return v;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    cudaError_t e = launch_quantize(W_bf16, d_out, d_in, group_size, symmetric, qweight,
+                                    static_cast<uint16_t*>(scales_fp16), static_cast<uint16_t*>(zeros_fp16), st.status,
+                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+wq_status wq_dequantize(const uint32_t* qweight, const void* scales_fp16, const void* zeros_fp16, int64_t d_out,
+                        int64_t d_in, int32_t group_size, int32_t symmetric, void* W_hat_bf16, void* stream) {
+    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
+    if (v != WQ_OK) return v;
+    if (!W_hat_bf16 || !aligned(W_hat_bf16, 16)) return WQ_ERR_INVALID_ARG;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    cudaError_t e = launch_dequantize(qweight, static_cast<const uint16_t*>(scales_fp16),
+                                      static_cast<const uint16_t*>(zeros_fp16), d_out, d_in, group_size, symmetric,
+                                      W_hat_bf16, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+size_t wq_linear_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in) {
+    (void)M;
+    (void)d_out;
+    (void)d_in;
+    return 0;
+}
+
+wq_status wq_linear_w4a16(const void* X_bf16, int64_t M, const uint32_t* qweight, const void* scales_fp16,
+                          const void* zeros_fp16, int64_t d_out, int64_t d_in, int32_t group_size, int32_t symmetric,
+                          void* Y, int32_t y_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
+    if (v != WQ_OK) return v;
+    if (!X_bf16 || !Y || !aligned(X_bf16, 16) || !aligned(Y, 16)) return WQ_ERR_INVALID_ARG;
+    if (M < 1 || M > (1ll << 31) - 1) return WQ_ERR_INVALID_ARG;
+    if (y_dtype != WQ_OUT_BF16 && y_dtype != WQ_OUT_FP32) return WQ_ERR_INVALID_ARG;
+    if (workspace_bytes < wq_linear_workspace_bytes(M, d_out, d_in)) return WQ_ERR_INVALID_ARG;
+    (void)workspace;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    LaunchOptions opt;
+    opt.pdl = pdl_enabled();
+    cudaError_t e;
+    if (M <= 16) {
+        GemvArgs a = {};
+        a.X = X_bf16;
+        a.scales = static_cast<const uint16_t*>(scales_fp16);
+        a.zeros = static_cast<const uint16_t*>(zeros_fp16);
+        a.Y = Y;
+        a.status = st.status;
+        a.M = (int)M;
+        a.N = (int)d_out;
+        a.K = (int)d_in;
+        a.g = group_size;
+        a.G = (int)(d_in / group_size);
+        a.symmetric = symmetric;
+        a.y_fp32 = y_dtype == WQ_OUT_FP32;
+        e = launch_gemv(qweight, a, st.num_sms, opt, s);
+    } else {
+        GemmArgs a = {};
+        a.X = X_bf16;
+        a.qweight = qweight;
+        a.scales = static_cast<const uint16_t*>(scales_fp16);
+        a.zeros = static_cast<const uint16_t*>(zeros_fp16);
+        a.Y = Y;
+        a.status = st.status;
+        a.M = (int)M;
+        a.N = (int)d_out;
+        a.K = (int)d_in;
+        a.g = group_size;
+        a.G = (int)(d_in / group_size);
+        a.symmetric = symmetric;
+        a.y_fp32 = y_dtype == WQ_OUT_FP32;
+        e = launch_gemm(a, st.num_sms, opt, s);
+    }
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+wq_status wq_selftest_bounded_wait(uint32_t limit_us, void* stream) {
+    if (limit_us < 1 || limit_us > 1000000) return WQ_ERR_INVALID_ARG;
+    DeviceState st;
+    wq_status v = device_state(&st);
+    if (v != WQ_OK) return v;
+    cudaError_t e = launch_bounded_wait_selftest(st.status, limit_us, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+wq_status wq_get_device_error(uint32_t* flags, void* stream) {
+    DeviceState st;
+    wq_status v = device_state(&st);
+    if (v != WQ_OK) return v;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t h = 0;
+    if (cudaMemcpyAsync(&h, st.status, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return WQ_ERR_CUDA;
+    if (cudaMemsetAsync(st.status, 0, sizeof(uint32_t), s) != cudaSuccess) return WQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return WQ_ERR_CUDA;
+    if (flags) *flags = h;
+    if (h & WQ_DEVFLAG_TIMEOUT) return WQ_ERR_TIMEOUT;
+    if (h & WQ_DEVFLAG_NONFINITE) return WQ_ERR_NONFINITE;
+    if (h & WQ_DEVFLAG_RANGE) return WQ_ERR_RANGE;
+    return WQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,63 @@
+// wq_kernels.h -- host-side launch functions of the libwq kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wq {
+
+cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric, uint32_t* qweight,
+                            uint16_t* scales, uint16_t* zeros, uint32_t* status, cudaStream_t stream);
+
+cudaError_t launch_dequantize(const uint32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
+                              int64_t d_out, int64_t d_in, int g, int symmetric, void* W_hat, cudaStream_t stream);
+
+// Decode GEMV, M <= 16.
+struct GemvArgs {
+    const void* X;           // bf16 [M][K]
+    const uint16_t* scales;  // fp16 [N][G]
+    const uint16_t* zeros;   // fp16 [N][G] or nullptr (symmetric)
+    void* Y;                 // [M][N] bf16 or fp32
+    uint32_t* status;
+    int M, N, K, G, g;
+    int rows_per_cta;  // npass * BR
+    int BR;            // rows per pass (TMA box height), <= 64
+    int npass;
+    int nkb;           // ceil(K / 128)
+    int nslots;        // smem ring slots
+    int slot_bytes;
+    int symmetric;
+    int y_fp32;
+};
+
+struct LaunchOptions {
+    bool pdl;  // programmatic dependent launch (prefetch weights before the previous kernel ends)
+};
+
+cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_sms, const LaunchOptions& opt,
+                        cudaStream_t stream);
+
+// Prefill GEMM on tcgen05 tensor cores, any M (used for M > 16).
+struct GemmArgs {
+    const void* X;           // bf16 [M][K]
+    const uint32_t* qweight; // [N][K/8]
+    const uint16_t* scales;  // fp16 [N][G]
+    const uint16_t* zeros;   // fp16 [N][G] or nullptr
+    void* Y;                 // [M][N]
+    uint32_t* status;
+    int M, N, K, G, g;
+    int symmetric;
+    int y_fp32;
+};
+
+cudaError_t launch_gemm(const GemmArgs& a, int num_sms, const LaunchOptions& opt, cudaStream_t stream);
+
+cudaError_t launch_bounded_wait_selftest(uint32_t* status, uint32_t limit_us, cudaStream_t stream);
+
+// Driver entry point for tensor-map encoding (resolved once through the runtime).
+CUresult encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                              uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                              CUtensorMapSwizzle swizzle);
+
+}  // namespace wq
