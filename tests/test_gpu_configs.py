@@ -3,7 +3,9 @@
 Configs 1-3 are checked completely (every code, scale, zero and output);
 configs 4 and 5 on sampled rows / outputs the oracle computes one by one,
 in the same launch configuration the benchmark times.  Packed artifacts are
-bit-exact; linear outputs satisfy |y - y_ref| <= 1e-3 * sum|w_hat x| + 1e-6."""
+bit-exact; linear outputs (bf16, as the benchmark runs them) satisfy the
+stated bound |y - y_ref| <= 1e-3 * sum|w_hat x| + 1e-6 as written, with no
+allowance for the output's own bf16 rounding."""
 import numpy as np
 import pytest
 import torch
@@ -13,6 +15,13 @@ from tests._util import bits16, bits32, linear_tolerance_ok
 from w4a16_bit_gemm_b200 import synthetic as syn
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clear_status():
+    from w4a16_bit_gemm_b200 import binding
+    binding.device_error()
+    yield
 
 
 def _b():
@@ -40,7 +49,7 @@ def check_full_case(wl, ci, Ms, device_gen="cpu"):
         X = syn.case_activations(wl, ci, M, device_gen)
         Y = b.linear_w4a16(X.cuda(), p)
         y_ref, A = oracle.linear(bits16(X), W_hat_ref)
-        ok, ratio = linear_tolerance_ok(Y.float().cpu().numpy(), y_ref, A)
+        ok, ratio = linear_tolerance_ok(Y.float().cpu().numpy(), y_ref, A, out_bf16=False)
         assert ok, (c.name, M, ratio)
 
 
@@ -81,7 +90,7 @@ def test_config4_prefill_sampled(ci):
         ridx = torch.from_numpy(rows).cuda()
         y = Y[ridx][:, idx].float().cpu().numpy()
         y_ref, A = oracle.linear(bits16(X[ridx]), W_hat_s)
-        ok, ratio = linear_tolerance_ok(y, y_ref, A)
+        ok, ratio = linear_tolerance_ok(y, y_ref, A, out_bf16=False)
         assert ok, (c.name, M, ratio)
         st, flags = b.device_error()
         assert st == b.WQ_OK
@@ -109,7 +118,7 @@ def test_config5_whole_model_sampled():
         X = syn.case_activations(wl, ci, 1, "cuda")
         Y = b.linear_w4a16(X, p)
         y_ref, A = oracle.linear(bits16(X), oracle.dequantize(codes, os_, oz, c.group_size))
-        ok, ratio = linear_tolerance_ok(Y[:, ridx].float().cpu().numpy(), y_ref, A)
+        ok, ratio = linear_tolerance_ok(Y[:, ridx].float().cpu().numpy(), y_ref, A, out_bf16=False)
         assert ok, (c.name, ratio)
         del W, p, X, Y
     payload, sb, zb = oracle.artifact_bytes(syn.total_params(wl), 4, 128, False)

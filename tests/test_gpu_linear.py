@@ -11,6 +11,13 @@ from tests._util import bits16, bf16_from_bits, f64_from_bf16_bits, linear_toler
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True)
+def _clear_status():
+    from w4a16_bit_gemm_b200 import binding
+    binding.device_error()
+    yield
+
+
 def _b():
     from w4a16_bit_gemm_b200 import binding
     return binding
@@ -37,7 +44,7 @@ def run_case(Wb, Xb, g, sym, out_dtype=torch.bfloat16, rows=None, cols=None):
     y_ref, A = oracle.linear(Xsel, W_hat)
     ysel = y if rows is None else y[rows]
     ysel = ysel if cols is None else ysel[:, cols]
-    ok, ratio = linear_tolerance_ok(ysel, y_ref, A)
+    ok, ratio = linear_tolerance_ok(ysel, y_ref, A, out_bf16=out_dtype == torch.bfloat16)
     assert ok, f"worst error/bound = {ratio:.3f}"
     return y, y_ref, A
 
@@ -51,7 +58,9 @@ GEMV_CASES = [
     (17, 1024, 64, False, 8),
     (260, 512, 512, False, 9),      # one group per row (per-channel scale)
     (5000, 1024, 128, False, 2),    # several rows per CTA
-    (40, 11008, 128, True, 4),      # long K
+    (40, 11008, 128, True, 4),      # long K, shared-memory ring (slots reused)
+    (20000, 2944, 128, False, 1),   # several passes per CTA, ring, 23 k blocks per pass
+    (4096, 11008, 128, True, 16),   # ring with two n-tiles
 ]
 
 

@@ -11,6 +11,13 @@ from tests._util import bits16, bits32, bf16_from_bits, fp16_from_bits
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True)
+def _clear_status():
+    from w4a16_bit_gemm_b200 import binding
+    binding.device_error()
+    yield
+
+
 def _binding():
     from w4a16_bit_gemm_b200 import binding
     return binding

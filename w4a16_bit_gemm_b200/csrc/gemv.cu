@@ -15,10 +15,11 @@
 //   memory slots; every slot has a "full" mbarrier (TMA transaction bytes) and
 //   an "empty" mbarrier (consumer releases).  When the CTA's whole share fits
 //   (the common decode case) every load is issued at kernel start.
-// - Consumer warps split the (k-block, 16-row tile) units of a pass.  A lane
-//   reads one 16-byte run (4 words = 32 k) of rows r and r+8 of a tile with one
-//   LDS.128 each: a quarter-warp reads two consecutive 64-byte rows, i.e. all
-//   32 banks once (conflict-free without swizzle).
+// - Consumer warp w takes chunks (k blocks) w, w+8, ... of a pass, all BR
+//   rows of each; a slot is always read by the same warp, so its phases are
+//   awaited in order.  A lane reads one 16-byte run (4 words = 32 k) of rows
+//   r and r+8 of a 16-row tile with one LDS.128 each: a quarter-warp reads two
+//   consecutive 64-byte rows, i.e. all 32 banks once (conflict-free).
 // - Nibbles are dequantized exactly in registers (bf16x2, see wq_device.cuh)
 //   straight into mma.sync m16n8k16 A fragments; the k order inside a
 //   fragment is permuted to match the nibble pairs (n, n+4) of a word, and the
@@ -100,10 +101,10 @@ __device__ __forceinline__ void load_bfrag(BFrag& f, const uint16_t* X, int K, i
     }
 }
 
-template <int NT>
+template <int NT, int TMAX>
 __global__ void __launch_bounds__(kGemvThreads, 1)
     gemv_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w, const GemvArgs a) {
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const GemvSmemLayout L = gemv_smem_layout(a);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
     uint64_t* empty = full + a.nslots;
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.nslots; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], (uint32_t)T);
+            mbar_init(&empty[i], 1u);
         }
         abort_flag = 0;
         fence_mbar_init();
@@ -177,79 +178,78 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
         }
         named_sync(1, nthreads_c);
 
-        float acc[4][NT][4];
+        float acc[TMAX][NT][4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
+        for (int t = 0; t < TMAX; ++t)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[t][nt][e] = 0.0f;
 
-        const int U = a.nkb * T;
-        const int u0 = warp * U / kGemvConsumerWarps, u1 = (warp + 1) * U / kGemvConsumerWarps;
-        int cached_kb = -1;
-        BFrag bf[NT];
-        for (int u = u0; u < u1; ++u) {
-            const int kb = u / T, tile = u - kb * T;
+        // Chunk c (one 128-wide k block, all BR rows; c counts across passes)
+        // belongs to consumer warp c % 8, and a ring's slot count is a multiple
+        // of 8, so every
+        // use of a slot is consumed by the same warp in order: a warp never
+        // waits on a slot phase that is two phases ahead of the barrier.
+        const int kb0 = (warp - (pass * a.nkb) % kGemvConsumerWarps + kGemvConsumerWarps) % kGemvConsumerWarps;
+        for (int kb = kb0; kb < a.nkb; kb += kGemvConsumerWarps) {
             const int c = pass * a.nkb + kb;
             const int slot = c % a.nslots;
             const int k0 = kb * kChunkK + 32 * tq;
             const bool kvalid = k0 < a.K;
-            if (kb != cached_kb) {
+            BFrag bf[NT];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) load_bfrag(bf[nt], X, a.K, a.M, nt * 8 + quad, k0, kvalid);
-                cached_kb = kb;
-            }
+            for (int nt = 0; nt < NT; ++nt) load_bfrag(bf[nt], X, a.K, a.M, nt * 8 + quad, k0, kvalid);
             const bool landed = mbar_wait(&full[slot], (uint32_t)(c / a.nslots) & 1u, a.status);
             if (!__all_sync(0xffffffffu, landed)) {  // warp-uniform give-up
                 if (lane == 0) atomicExch(&abort_flag, 1);
                 break;
             }
             const uint8_t* sp = slots + (size_t)slot * a.slot_bytes;
-            const int ra = tile * 16 + quad, rb = ra + 8;
-            uint32_t pa[4][4], pb[4][4];
-            if (kvalid) {
-                const int gcol = k0 / a.g;
-                uint4 wa = make_uint4(0, 0, 0, 0), wb = make_uint4(0, 0, 0, 0);
-                if (ra < a.BR) wa = *reinterpret_cast<const uint4*>(sp + ra * kChunkRowBytes + tq * 16);
-                if (rb < a.BR) wb = *reinterpret_cast<const uint4*>(sp + rb * kChunkRowBytes + tq * 16);
-                const int ia = min(ra, a.BR - 1) * a.G + gcol, ib = min(rb, a.BR - 1) * a.G + gcol;
-                const GroupConsts ca = make_group_consts(sz_s[ia], sym ? 0 : (int)__half2float(__ushort_as_half(sz_z[ia])), sym);
-                const GroupConsts cb = make_group_consts(sz_s[ib], sym ? 0 : (int)__half2float(__ushort_as_half(sz_z[ib])), sym);
-                const uint32_t wav[4] = {wa.x, wa.y, wa.z, wa.w}, wbv[4] = {wb.x, wb.y, wb.z, wb.w};
+            const int gcol = kvalid ? k0 / a.g : 0;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    dequant_word_pairs(wav[j], ca, pa[j]);
-                    dequant_word_pairs(wbv[j], cb, pb[j]);
+            for (int t = 0; t < TMAX; ++t) {
+                if (t >= T) break;
+                const int ra = t * 16 + quad, rb = ra + 8;
+                uint32_t pa[4][4], pb[4][4];
+                if (kvalid) {
+                    uint4 wa = make_uint4(0, 0, 0, 0), wb = make_uint4(0, 0, 0, 0);
+                    if (ra < a.BR) wa = *reinterpret_cast<const uint4*>(sp + ra * kChunkRowBytes + tq * 16);
+                    if (rb < a.BR) wb = *reinterpret_cast<const uint4*>(sp + rb * kChunkRowBytes + tq * 16);
+                    const int ia = min(ra, a.BR - 1) * a.G + gcol, ib = min(rb, a.BR - 1) * a.G + gcol;
+                    const GroupConsts ca =
+                        make_group_consts(sz_s[ia], sym ? 0 : (int)__half2float(__ushort_as_half(sz_z[ia])), sym);
+                    const GroupConsts cb =
+                        make_group_consts(sz_s[ib], sym ? 0 : (int)__half2float(__ushort_as_half(sz_z[ib])), sym);
+                    const uint32_t wav[4] = {wa.x, wa.y, wa.z, wa.w}, wbv[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        dequant_word_pairs(wav[j], ca, pa[j]);
+                        dequant_word_pairs(wbv[j], cb, pb[j]);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) pa[j][p] = pb[j][p] = 0u;
                 }
-            } else {
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
+                for (int i = 0; i < 8; ++i) {
+                    const int j = i / 2, p = 2 * (i % 2);
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) pa[j][p] = pb[j][p] = 0u;
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816(acc[t][nt], pa[j][p], pb[j][p], pa[j][p + 1], pb[j][p + 1], bf[nt].b01[i],
+                                  bf[nt].b23[i]);
+                }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);  // smem slot no longer read by this warp
-
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                if (t == tile) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int j = i / 2, p = 2 * (i % 2);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_16816(acc[t][nt], pa[j][p], pb[j][p], pa[j][p + 1], pb[j][p + 1], bf[nt].b01[i],
-                                      bf[nt].b23[i]);
-                    }
-                }
-            }
+            if (lane == 0) mbar_arrive(&empty[slot]);  // this warp is the slot's only reader
         }
 
         // ---- deterministic reduction over consumer warps ----
         const int T16 = T * 16;
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
+        for (int t = 0; t < TMAX; ++t) {
             if (t < T) {
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
@@ -306,11 +306,18 @@ cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_s
     a.nslots = 1;
     GemvSmemLayout L = gemv_smem_layout(a);
     const int fixed = L.slot_off;
-    int nslots = (budget - fixed) / a.slot_bytes;
+    const int nslots_fit = (budget - fixed) / a.slot_bytes;
     const int total_chunks = a.npass * a.nkb;
-    if (nslots > total_chunks) nslots = total_chunks;
-    if (nslots > 64) nslots = 64;
-    if (nslots < 2) nslots = 2;
+    int nslots;
+    if (nslots_fit >= total_chunks && total_chunks <= 64) {
+        nslots = total_chunks;  // whole share resident: every slot used once
+    } else {
+        // ring: every slot is owned by one consumer warp, so the count is a
+        // multiple of the warp count
+        nslots = nslots_fit < 64 ? nslots_fit : 64;
+        nslots = nslots / kGemvConsumerWarps * kGemvConsumerWarps;
+        if (nslots < kGemvConsumerWarps) return cudaErrorInvalidConfiguration;
+    }
     a.nslots = nslots;
     L = gemv_smem_layout(a);
     if (L.total > 220 * 1024) return cudaErrorInvalidConfiguration;
@@ -321,7 +328,7 @@ cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_s
                                        CU_TENSOR_MAP_SWIZZLE_NONE);
     if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
-    void (*kern)(const CUtensorMap, const GemvArgs) = NT == 1 ? gemv_w4a16_kernel<1> : gemv_w4a16_kernel<2>;
+    void (*kern)(const CUtensorMap, const GemvArgs) = NT == 1 ? gemv_w4a16_kernel<1, 4> : gemv_w4a16_kernel<2, 2>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
     if (e != cudaSuccess) return e;
 
