@@ -162,3 +162,14 @@ def test_bounded_wait_selftest_sets_timeout():
     b.linear_w4a16(torch.randn(1, 256, device="cuda").to(torch.bfloat16), p)
     st, flags = b.device_error()
     assert st == b.WQ_OK and flags == 0
+
+
+def test_gemv_m1_large_rows_fallback():
+    """A single-token GEMV whose per-CTA constants exceed the resident plan
+    (many rows per SM) takes the MMA kernel; still within the bound."""
+    rng = np.random.default_rng(21)
+    N, K = 28672, 1024
+    W = bf16_bits_of(rng.standard_normal((N, K)) * 0.02)
+    X = bf16_bits_of(rng.standard_normal((1, K)))
+    cols = np.sort(rng.choice(N, 300, replace=False))
+    run_case(W, X, 128, False, torch.float32, cols=cols)

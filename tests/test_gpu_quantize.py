@@ -144,3 +144,31 @@ def test_dequantize_exhaustive_scale_code_zero(sym):
                        None if sym else fp16_from_bits(zeros).cuda(), d_out, d_in, g, sym)
     out = b.dequantize(P)
     assert np.array_equal(bits16(out), ref)
+
+
+def _all_bf16_between(lo, hi):
+    u = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):
+        v = (u.astype(np.uint32) << 16).view(np.float32)
+    keep = np.isfinite(v) & (v >= lo) & (v <= hi)
+    return u[keep]
+
+
+@pytest.mark.parametrize("lo,hi,sym", [
+    (-1.0, 1.5, False), (-0.0625, 0.75, False), (-3.0, -0.5, False), (0.25, 7.0, False),
+    (-0.5, 0.5, True), (-2.0, 0.75, True), (-1e-3, 2e-2, False), (-65000.0, 1.0, False),
+])
+def test_every_bf16_in_window(lo, hi, sym):
+    """Each group holds the window ends plus 30 values; together the groups
+    cover every bf16 value in the window, so every quotient near a
+    half-integer (the exact-division fallback) is exercised."""
+    g = 32
+    pool = _all_bf16_between(lo, hi)
+    ends = bf16_bits_of([lo, hi])
+    n_grp = -(-len(pool) // (g - 2))
+    free = np.resize(pool, n_grp * (g - 2)).reshape(n_grp, g - 2)
+    W = np.concatenate([np.repeat(ends[None, :], n_grp, 0), free], axis=1)
+    # several groups per row
+    rows = -(-n_grp // 8)
+    W = np.resize(W, (rows * 8, g)).reshape(rows, 8 * g)
+    check_quantize(np.ascontiguousarray(W), g, sym)

@@ -121,7 +121,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                               const GemmArgs a) {
     using SL = GemmSmem<MSUB>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // the dynamic shared-memory base is only guaranteed 16-byte alignment; the
+    // 128-byte swizzle atoms need 1024 (the launch adds 1024 bytes of slack)
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full1 = reinterpret_cast<uint64_t*>(smem + SL::kOffBar);
     uint64_t* empty1 = full1 + kS1;
     uint64_t* full2 = empty1 + kS1;

@@ -72,9 +72,24 @@ __device__ __forceinline__ ScaleZero scale_zero(float lo, float hi, bool symmetr
     return r;
 }
 
+// rint(x / s) for the IEEE-rounded quotient, without a division on the fast
+// path.  f = x * rcp_rn(s) differs from x/s by at most (2^-23 + 2^-48)|x/s|
+// and the rounded quotient fl(x/s) by at most 2^-24|x/s|, so for |f| < 32
+// the two lie within 3 * 2^-24 * 32 < 2^-17 of each other: when f is more
+// than 2^-17 away from the nearest half-integer both round to the same
+// integer.  Otherwise the exact IEEE division decides.  For |f| >= 32 the
+// code is clamped to the same end of the range either way (|q - z| <= 15).
+__device__ __forceinline__ float rint_quotient(float x, float s, float rcp) {
+    const float f = __fmul_rn(x, rcp);
+    float t = rintf(f);
+    if (fabsf(f) < 32.0f && fabsf(__fsub_rn(f, t)) > 0.5f - 0x1p-17f) t = rintf(__fdiv_rn(x, s));
+    return t;
+}
+
 // Codes of 8 weights packed into one word (low nibble first).
 __device__ __forceinline__ uint32_t encode8(const float v[8], const ScaleZero& sz, bool symmetric) {
     const float s = __half2float(__ushort_as_half(sz.s16));
+    const float rcp = __frcp_rn(s);
     const float qmin = symmetric ? -8.0f : 0.0f;
     const float qmax = symmetric ? 7.0f : 15.0f;
     const float zf = (float)sz.z;
@@ -85,8 +100,8 @@ __device__ __forceinline__ uint32_t encode8(const float v[8], const ScaleZero& s
         if (isnan(v[i])) {
             q = sz.z;
         } else {
-            float t = rintf(__fdiv_rn(v[i], s));
-            float c = fminf(fmaxf(__fadd_rn(t, zf), qmin), qmax);
+            const float t = rint_quotient(v[i], s, rcp);
+            const float c = fminf(fmaxf(__fadd_rn(t, zf), qmin), qmax);
             q = (int)c;
         }
         word |= ((uint32_t)q & 0xfu) << (4 * i);
@@ -94,8 +109,9 @@ __device__ __forceinline__ uint32_t encode8(const float v[8], const ScaleZero& s
     return word;
 }
 
-// g <= 256: L = g/8 lanes per group, 32/L groups per warp; each thread does
-// kSegPerThread segments spaced one block-width apart (loads issued first).
+// g <= 256: L = g/8 lanes per group, 32/L groups per warp.  Grid-stride:
+// each thread handles kSegPerThread segments spaced one block-width apart per
+// iteration, all loads issued before any arithmetic.
 constexpr int kQuantThreads = 256;
 constexpr int kSegPerThread = 2;
 
@@ -104,39 +120,42 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_small_group_kernel(
     const uint4* __restrict__ W, int64_t nseg, int symmetric, uint32_t* __restrict__ qweight,
     uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros, uint32_t* status) {
     const int lane = threadIdx.x & 31;
-    const int64_t base = (int64_t)blockIdx.x * (kQuantThreads * kSegPerThread) + threadIdx.x;
-    uint4 raw[kSegPerThread];
-#pragma unroll
-    for (int u = 0; u < kSegPerThread; ++u) {
-        int64_t seg = base + (int64_t)u * kQuantThreads;
-        raw[u] = seg < nseg ? ld_nc_v4(W + seg) : make_uint4(0, 0, 0, 0);
-    }
     bool nonfinite = false, range = false;
+    const int64_t stride = (int64_t)gridDim.x * (kQuantThreads * kSegPerThread);
+    for (int64_t base = (int64_t)blockIdx.x * (kQuantThreads * kSegPerThread) + threadIdx.x; base - threadIdx.x < nseg;
+         base += stride) {
+        uint4 raw[kSegPerThread];
 #pragma unroll
-    for (int u = 0; u < kSegPerThread; ++u) {
-        const int64_t seg = base + (int64_t)u * kQuantThreads;
-        float v[8];
-        unpack_bf16x8(raw[u], v);
-        float lo = 0.0f, hi = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            nonfinite |= !isfinite(v[i]);
-            lo = fminf(lo, v[i]);
-            hi = fmaxf(hi, v[i]);
+        for (int u = 0; u < kSegPerThread; ++u) {
+            const int64_t seg = base + (int64_t)u * kQuantThreads;
+            raw[u] = seg < nseg ? ld_nc_v4(W + seg) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int o = 1; o < L; o <<= 1) {
-            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-        }
-        ScaleZero sz = scale_zero(lo, hi, symmetric != 0);
-        if (seg < nseg) {
-            range |= sz.range;
-            qweight[seg] = encode8(v, sz, symmetric != 0);
-            if ((lane & (L - 1)) == 0) {
-                const int64_t gi = seg / L;
-                scales[gi] = sz.s16;
-                if (!symmetric) zeros[gi] = __half_as_ushort(__int2half_rn(sz.z));
+        for (int u = 0; u < kSegPerThread; ++u) {
+            const int64_t seg = base + (int64_t)u * kQuantThreads;
+            float v[8];
+            unpack_bf16x8(raw[u], v);
+            float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                nonfinite |= !isfinite(v[i]);
+                lo = fminf(lo, v[i]);
+                hi = fmaxf(hi, v[i]);
+            }
+#pragma unroll
+            for (int o = 1; o < L; o <<= 1) {
+                lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+            }
+            ScaleZero sz = scale_zero(lo, hi, symmetric != 0);
+            if (seg < nseg) {
+                range |= sz.range;
+                qweight[seg] = encode8(v, sz, symmetric != 0);
+                if ((lane & (L - 1)) == 0) {
+                    const int64_t gi = seg / L;
+                    scales[gi] = sz.s16;
+                    if (!symmetric) zeros[gi] = __half_as_ushort(__int2half_rn(sz.z));
+                }
             }
         }
     }
@@ -189,40 +208,57 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_large_group_kernel(
 
 // Dequantize: each thread expands 4 packed words (32 weights of one group)
 // into 64 bytes of bf16, using the exact bf16x2 dequantization shared with the
-// linear-layer kernels.
+// linear-layer kernels.  Grid-stride with two quads in flight per thread.
 constexpr int kDeqThreads = 256;
+constexpr int kDeqPerThread = 2;
 
 __global__ void __launch_bounds__(kDeqThreads) dequantize_kernel(
     const uint4* __restrict__ qweight, const uint16_t* __restrict__ scales,
     const uint16_t* __restrict__ zeros, int64_t nquad, int g, int symmetric, uint4* __restrict__ W_hat) {
-    const int64_t t = (int64_t)blockIdx.x * kDeqThreads + threadIdx.x;
-    if (t >= nquad) return;
-    const uint4 q = ld_nc_v4(qweight + t);
-    const int64_t gi = (t * 32) / g;
-    const uint16_t s16 = scales[gi];
-    int z = 0;
-    if (!symmetric) z = (int)__half2float(__ushort_as_half(zeros[gi]));
-    const GroupConsts c = make_group_consts(s16, z, symmetric != 0);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    const int64_t stride = (int64_t)gridDim.x * (kDeqThreads * kDeqPerThread);
+    for (int64_t base = (int64_t)blockIdx.x * (kDeqThreads * kDeqPerThread) + threadIdx.x; base < nquad;
+         base += stride) {
+        uint4 q[kDeqPerThread];
+        uint16_t s16[kDeqPerThread], z16[kDeqPerThread];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        uint32_t o[4];
-        dequant_word_natural(w[j], c, o);
-        W_hat[t * 4 + j] = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int u = 0; u < kDeqPerThread; ++u) {
+            const int64_t t = base + (int64_t)u * kDeqThreads;
+            if (t < nquad) {
+                q[u] = ld_nc_v4(qweight + t);
+                const int64_t gi = (t * 32) / g;
+                s16[u] = scales[gi];
+                z16[u] = symmetric ? (uint16_t)0 : zeros[gi];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kDeqPerThread; ++u) {
+            const int64_t t = base + (int64_t)u * kDeqThreads;
+            if (t >= nquad) continue;
+            const int z = symmetric ? 0 : (int)__half2float(__ushort_as_half(z16[u]));
+            const GroupConsts c = make_group_consts(s16[u], z, symmetric != 0);
+            const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t o[4];
+                dequant_word_natural(w[j], c, o);
+                W_hat[t * 4 + j] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
     }
 }
 
 }  // namespace
 
 cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric,
-                            uint32_t* qweight, uint16_t* scales, uint16_t* zeros, uint32_t* status,
+                            uint32_t* qweight, uint16_t* scales, uint16_t* zeros, uint32_t* status, int num_sms,
                             cudaStream_t stream) {
     const int64_t P = d_out * d_in;
     const uint4* W4 = static_cast<const uint4*>(W);
     if (g <= 256) {
         const int64_t nseg = P / 8;
         const int64_t per_block = (int64_t)kQuantThreads * kSegPerThread;
-        const int64_t blocks = (nseg + per_block - 1) / per_block;
+        int64_t blocks = (nseg + per_block - 1) / per_block;
+        if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
         switch (g) {
             case 32:
                 quantize_small_group_kernel<4><<<blocks, kQuantThreads, 0, stream>>>(W4, nseg, symmetric, qweight,
@@ -254,10 +290,11 @@ cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, i
 }
 
 cudaError_t launch_dequantize(const uint32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
-                              int64_t d_out, int64_t d_in, int g, int symmetric, void* W_hat,
+                              int64_t d_out, int64_t d_in, int g, int symmetric, void* W_hat, int num_sms,
                               cudaStream_t stream) {
     const int64_t nquad = d_out * d_in / 32;
-    const int64_t blocks = (nquad + kDeqThreads - 1) / kDeqThreads;
+    int64_t blocks = (nquad + kDeqThreads * kDeqPerThread - 1) / (kDeqThreads * kDeqPerThread);
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
     dequantize_kernel<<<blocks, kDeqThreads, 0, stream>>>(reinterpret_cast<const uint4*>(qweight), scales, zeros,
                                                           nquad, g, symmetric, static_cast<uint4*>(W_hat));
     return cudaGetLastError();

@@ -142,7 +142,7 @@ wq_status wq_quantize_rtn(const void* W_bf16, int64_t d_out, int64_t d_in, int32
     if ((v = device_state(&st)) != WQ_OK) return v;
     cudaError_t e = launch_quantize(W_bf16, d_out, d_in, group_size, symmetric, qweight,
                                     static_cast<uint16_t*>(scales_fp16), static_cast<uint16_t*>(zeros_fp16), st.status,
-                                    static_cast<cudaStream_t>(stream));
+                                    st.num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
@@ -155,7 +155,7 @@ wq_status wq_dequantize(const uint32_t* qweight, const void* scales_fp16, const 
     if ((v = device_state(&st)) != WQ_OK) return v;
     cudaError_t e = launch_dequantize(qweight, static_cast<const uint16_t*>(scales_fp16),
                                       static_cast<const uint16_t*>(zeros_fp16), d_out, d_in, group_size, symmetric,
-                                      W_hat_bf16, static_cast<cudaStream_t>(stream));
+                                      W_hat_bf16, st.num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
@@ -194,6 +194,9 @@ wq_status wq_linear_w4a16(const void* X_bf16, int64_t M, const uint32_t* qweight
         a.K = (int)d_in;
         a.g = group_size;
         a.G = (int)(d_in / group_size);
+        a.g_shift = -1;
+        for (int sh = 0; sh < 31; ++sh)
+            if ((1 << sh) == group_size) a.g_shift = sh;
         a.symmetric = symmetric;
         a.y_fp32 = y_dtype == WQ_OUT_FP32;
         e = launch_gemv(qweight, a, st.num_sms, opt, s);

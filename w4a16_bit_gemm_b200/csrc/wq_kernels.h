@@ -8,10 +8,11 @@
 namespace wq {
 
 cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric, uint32_t* qweight,
-                            uint16_t* scales, uint16_t* zeros, uint32_t* status, cudaStream_t stream);
+                            uint16_t* scales, uint16_t* zeros, uint32_t* status, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_dequantize(const uint32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
-                              int64_t d_out, int64_t d_in, int g, int symmetric, void* W_hat, cudaStream_t stream);
+                              int64_t d_out, int64_t d_in, int g, int symmetric, void* W_hat, int num_sms,
+                              cudaStream_t stream);
 
 // Decode GEMV, M <= 16.
 struct GemvArgs {
@@ -21,12 +22,18 @@ struct GemvArgs {
     void* Y;                 // [M][N] bf16 or fp32
     uint32_t* status;
     int M, N, K, G, g;
+    int g_shift;       // log2(g) when g is a power of two, else -1
     int rows_per_cta;  // npass * BR
-    int BR;            // rows per pass (TMA box height), <= 64
+    int BR;            // rows per pass, <= 64
+    int T;             // tiles per pass
+    int BRT;           // rows per tile (TMA box height), <= 16
     int npass;
     int nkb;           // ceil(K / 128)
-    int nslots;        // smem ring slots
+    int nks;           // row segments of 2048 k per row
+    int pitch;         // padded shared-memory row pitch of a slot (bytes)
+    int nslots;        // smem slots (ring when fewer than the chunks)
     int slot_bytes;
+    int xs_bytes;      // activations staged in smem (0: read from global)
     int symmetric;
     int y_fp32;
 };
