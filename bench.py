@@ -52,6 +52,31 @@ def quant_bytes(N: int, K: int, symmetric: bool, g: int = 128) -> int:
     return N * K * 2 + N * K // 2 + (N * K // g) * per_group
 
 
+def source_digest() -> str:
+    """sha256 over the CUDA sources; DRAM counters taken from an older build do not apply."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "w4a16_bit_gemm_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def kernel_traffic(name: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when it is
+    missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", name)
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_sha256") != source_digest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -331,14 +356,7 @@ def run_ours(args, dist: Dist):
     if st != b.WQ_OK:
         raise RuntimeError(f"device status after the bench: {st} flags {flags}")
 
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "gemv_traffic.json")
-    if os.path.exists(tpath):
-        try:
-            with open(tpath) as f:
-                traffic = json.load(f).get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = kernel_traffic("gemv_traffic.json")
 
     out = {
         "metric": METRIC,

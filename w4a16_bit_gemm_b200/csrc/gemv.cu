@@ -405,8 +405,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 // M = 1: CUDA-core dot product.  The m16n8k16 MMA would waste 7/8 of its
 // n dimension on one token, so the single-token GEMV multiplies on the FMA
 // pipe instead: fma.rn.f32.bf16 takes the exact bf16 x_hat and the bf16
-// activation as operands and accumulates in fp32 (one rounding per product,
-// as an fp32 FFMA of the widened values).
+// activation as operands and accumulates in fp32 (one rounding per product
+// and accumulation, as an fp32 FFMA of the widened values).
 // - A CTA's rows are one contiguous byte range of qweight, so the producer
 //   moves them with 1D bulk copies of <= 16 KB (the copy engine streams these
 //   at HBM rate; many small row pieces it cannot).  A chunk is RC consecutive
@@ -414,7 +414,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 //   where every consumer warp consumes every chunk in order.
 // - A unit is (row, 1024-k part): lane l takes the 32-k slice l of the part
 //   (4 packed words, one LDS.128; a warp reads 512 contiguous bytes).  Units
-//   are dealt round-robin to 16 consumer warps, so rows need no padding.
+//   are dealt round-robin to 16 consumer warps, so rows need no padding; a
+//   warp keeps its activation slice (fp32) in registers while its part
+//   repeats.
 // - Each unit's 32 lane partials are folded to 8 with two shuffles and
 //   parked in shared memory; a fixed-order sum per row finishes (deterministic).
 // ------------------------------------------------------------------------
@@ -561,16 +563,20 @@ __global__ void __launch_bounds__(kM1Threads, 1)
         }
         const uint32_t xw[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
                                  v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
-        uint32_t o[16];
+        uint32_t pw[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            o[4 * j + 0] = __byte_perm(xw[4 * j], xw[4 * j + 2], 0x5410);
-            o[4 * j + 1] = __byte_perm(xw[4 * j], xw[4 * j + 2], 0x7632);
-            o[4 * j + 2] = __byte_perm(xw[4 * j + 1], xw[4 * j + 3], 0x5410);
-            o[4 * j + 3] = __byte_perm(xw[4 * j + 1], xw[4 * j + 3], 0x7632);
-        }
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) xs[it * 4 + q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            for (int p = 0; p < 4; ++p) {
+                // element e of the slice sits in half (e & 1) of word e >> 1
+                const int e0 = 8 * j + p, e1 = 8 * j + p + 4;
+                const uint32_t lo = (e0 & 1) ? (xw[e0 >> 1] >> 16) : (xw[e0 >> 1] & 0xffffu);
+                const uint32_t hi = (e1 & 1) ? (xw[e1 >> 1] & 0xffff0000u) : (xw[e1 >> 1] << 16);
+                pw[4 * j + p] = lo | hi;
+            }
+        uint4* dst = xs + it * 4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
     }
     for (int i = threadIdx.x + kPf * nthreads_c; i < nitems; i += nthreads_c) {
         const int64_t gi = (int64_t)row0 * a.G + i;
@@ -598,7 +604,7 @@ __global__ void __launch_bounds__(kM1Threads, 1)
         for (int u = warp; u < rows * nkp; u += kM1Warps) {
             const int r = c * RC + rl;  // CTA row
             const int s = kp * 32 + lane;
-            float acc0 = 0.0f, acc1 = 0.0f;
+            float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
             if (s < nsl) {
                 const int k0 = s * 32;
                 if (kp != cached_kp) {  // the activation slice stays in registers while kp repeats
@@ -617,11 +623,13 @@ __global__ void __launch_bounds__(kM1Threads, 1)
                 for (int j = 0; j < 4; ++j) {
                     uint32_t pr[4];
                     dequant_word_pairs(wv[j], gc, pr);
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) fma2_bf16_f32(acc0, acc1, pr[p], xr[4 * j + p]);
+                    fma2_bf16_f32(a0, a1, pr[0], xr[4 * j + 0]);
+                    fma2_bf16_f32(a2, a3, pr[1], xr[4 * j + 1]);
+                    fma2_bf16_f32(a0, a1, pr[2], xr[4 * j + 2]);
+                    fma2_bf16_f32(a2, a3, pr[3], xr[4 * j + 3]);
                 }
             }
-            float v = acc0 + acc1;
+            float v = (a0 + a1) + (a2 + a3);
             v += __shfl_xor_sync(0xffffffffu, v, 16);
             v += __shfl_xor_sync(0xffffffffu, v, 8);
             if (lane < 8) red[(r * nkp + kp) * 8 + lane] = v;
@@ -636,11 +644,14 @@ __global__ void __launch_bounds__(kM1Threads, 1)
         if (lane == 0) mbar_arrive(&empty[slot]);
     }
     named_sync(1, nthreads_c);
-    // fixed-order sum of each row's parked partials
-    for (int r = threadIdx.x; r < nrows; r += nthreads_c) {
+    // each row's parked partials summed by one warp: lane-strided partial sums,
+    // then a shuffle tree (a fixed order, so the result is deterministic)
+    for (int r = warp; r < nrows; r += kM1Warps) {
         float v = 0.0f;
-        for (int q = 0; q < nkp * 8; ++q) v += red[r * nkp * 8 + q];
-        if (!abort_flag) {
+        for (int q = lane; q < nkp * 8; q += 32) v += red[r * nkp * 8 + q];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && !abort_flag) {
             if (a.y_fp32)
                 static_cast<float*>(a.Y)[row0 + r] = v;
             else
