@@ -61,6 +61,14 @@ GEMV_CASES = [
     (40, 11008, 128, True, 4),      # long K, shared-memory ring (slots reused)
     (20000, 2944, 128, False, 1),   # several passes per CTA, ring, 23 k blocks per pass
     (4096, 11008, 128, True, 16),   # ring with two n-tiles
+    # tensor-memory GEMV (M = 2, or M = 1 with K >= 8192; K % 256 == 0): ragged
+    # row counts per CTA, several 32-row MMA tiles per CTA, every group size
+    (333, 2048, 32, False, 2),
+    (10360, 1024, 64, True, 2),     # 70 rows per CTA: three tiles of 24/23/23
+    (2000, 512, 256, False, 2),
+    (29600, 256, 128, False, 2),    # 200 rows per CTA, capped at 128: more CTAs than SMs
+    (40000, 256, 128, True, 2),
+    (700, 8192, 128, False, 1),     # M = 1, long rows: tensor-memory kernel
 ]
 
 

@@ -87,9 +87,6 @@ __device__ __forceinline__ void mma_16816(float c[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // B fragments of one 128-wide k block for token n: the lane's 32 k values
 // (k0 .. k0+31), paired to match dequant_word_pairs: MMA i takes
@@ -148,20 +145,6 @@ __device__ __forceinline__ void store_xs(uint4* xs, int M, int kb, int n, int t4
 }
 
 // 8-byte packed constants -> the four bf16x2 words of GroupConsts.
-__device__ __forceinline__ GroupConsts unpack_consts(uint2 v) {
-    GroupConsts c;
-    c.s_hi = __byte_perm(v.x, v.x, 0x1010);
-    c.s_lo = __byte_perm(v.x, v.x, 0x3232);
-    c.zm = __byte_perm(v.y, v.y, 0x1010);
-    c.xmask = __byte_perm(v.y, v.y, 0x3232);
-    return c;
-}
-
-__device__ __forceinline__ uint2 pack_consts(uint16_t s16, int z, bool sym) {
-    const GroupConsts g = make_group_consts(s16, z, sym);
-    return make_uint2((g.s_hi & 0xffffu) | (g.s_lo << 16), (g.zm & 0xffffu) | (g.xmask << 16));
-}
-
 // NCH independent accumulator chains per warp: consecutive MMAs of a unit go
 // to different chains, so the MMA result latency is not on the critical path.
 template <int NT, int NCH>
@@ -761,7 +744,20 @@ cudaError_t launch_gemv_variant(const uint32_t* qweight, GemvArgs a, int num_sms
 
 cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_sms, const LaunchOptions& opt,
                         cudaStream_t stream) {
-    if (base.M == 1) {
+    // M = 1 with rows up to 8K k: the CUDA-core kernel is the faster one (measured
+    // 7.0 vs 9.0 us at 4096x4096, 14.7 vs 18.4 us at 11008x4096); longer rows and
+    // M = 2 run faster on the tensor-memory kernel (15.7 vs 17.6 us at 4096x11008,
+    // M = 2: 9.1 vs 10.6 us at 4096x4096).
+    const bool m1_first = base.M == 1 && base.K < 8192;
+    if (m1_first) {
+        const cudaError_t e = launch_gemv_m1(qweight, base, num_sms, opt, stream);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    if (base.M <= 2 && !gemv_tc_disabled()) {
+        const cudaError_t e = launch_gemv_tc(qweight, base, num_sms, opt, stream);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    if (base.M == 1 && !m1_first) {
         const cudaError_t e = launch_gemv_m1(qweight, base, num_sms, opt, stream);
         if (e != cudaErrorNotSupported) return e;
     }

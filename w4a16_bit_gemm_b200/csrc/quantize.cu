@@ -72,6 +72,54 @@ __device__ __forceinline__ ScaleZero scale_zero(float lo, float hi, bool symmetr
     return r;
 }
 
+// rcp.approx.f32: at most 1 ulp from 1/s.
+__device__ __forceinline__ float rcp_approx(float s) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(s));
+    return r;
+}
+
+// rint(fl32(-lo / s)) with the IEEE division (rare: near a half-integer).
+__device__ __noinline__ float exact_neg_quotient_rint(float lo, float s) {
+    return rintf(__fsub_rn(0.0f, __fdiv_rn(lo, s)));
+}
+
+// scale_zero without fp32 divisions on the common path.
+//  - fl32(r / 15) (or / 7) equals fl32(fl64(r) * fl64(1/15)): r has 24
+//    significant bits, so a quotient that is not exact lies at least 2^-29
+//    (relative) away from every fp32 rounding midpoint, while the fp64
+//    product is within 2^-52 of the quotient (correct rounding of the
+//    quotient is preserved).
+//  - z = rint(fl32(-lo / s)) through f = -lo * rcp(s) with the quotient
+//    guard of rint_quotient (the exact division decides near a half-integer).
+// Also returns rcp(s) for the code path.
+__device__ __forceinline__ ScaleZero scale_zero_fast(float lo, float hi, bool symmetric, float& rcp_out) {
+    float s32;
+    if (symmetric)
+        s32 = __double2float_rn((double)fmaxf(-lo, hi) * (1.0 / 7.0));
+    else
+        s32 = __double2float_rn((double)__fsub_rn(hi, lo) * (1.0 / 15.0));
+    ScaleZero r;
+    r.s16 = __half_as_ushort(__float2half_rn(s32));
+    r.range = false;
+    r.z = 0;
+    if (r.s16 == 0x7c00u) {  // fp16 overflow: saturate
+        r.s16 = 0x7bffu;
+        r.range = true;
+    }
+    if (r.s16 == 0u) r.s16 = 0x3c00u;  // all-zero or underflowing group
+    const float s = __half2float(__ushort_as_half(r.s16));
+    const float rcp = rcp_approx(s);
+    rcp_out = rcp;
+    if (!symmetric && lo != 0.0f) {
+        const float f = __fmul_rn(-lo, rcp);
+        float t = rintf(f);
+        if (fabsf(f) < 32.0f && fabsf(__fsub_rn(f, t)) > 0.5f - 0x1p-17f) t = exact_neg_quotient_rint(lo, s);
+        r.z = (int)fminf(fmaxf(t, 0.0f), 15.0f);
+    }
+    return r;
+}
+
 // rint(x / s) for the IEEE-rounded quotient, without a division on the fast
 // path.  f = x * rcp_rn(s) differs from x/s by at most (2^-23 + 2^-48)|x/s|
 // and the rounded quotient fl(x/s) by at most 2^-24|x/s|, so for |f| < 32
@@ -87,6 +135,8 @@ __device__ __forceinline__ float rint_quotient(float x, float s, float rcp) {
 }
 
 // Codes of 8 weights packed into one word (low nibble first).
+__device__ __noinline__ uint32_t encode8_slow(const uint4 raw, const ScaleZero sz, bool symmetric);
+
 __device__ __forceinline__ uint32_t encode8(const float v[8], const ScaleZero& sz, bool symmetric) {
     const float s = __half2float(__ushort_as_half(sz.s16));
     const float rcp = __frcp_rn(s);
@@ -109,52 +159,175 @@ __device__ __forceinline__ uint32_t encode8(const float v[8], const ScaleZero& s
     return word;
 }
 
-// g <= 256: L = g/8 lanes per group, 32/L groups per warp.  Grid-stride:
-// each thread handles kSegPerThread segments spaced one block-width apart per
-// iteration, all loads issued before any arithmetic.
 constexpr int kQuantThreads = 256;
-constexpr int kSegPerThread = 2;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+
+// Statistics of 32 values skipping NaN (rare: only threads that hold a NaN).
+__device__ __noinline__ float2 nan_skipping_min_max(const uint4 r0, const uint4 r1, const uint4 r2, const uint4 r3) {
+    const uint4 rr[4] = {r0, r1, r2, r3};
+    float lo = 0.0f, hi = 0.0f;
+    for (int v = 0; v < 4; ++v) {
+        float f[8];
+        unpack_bf16x8(rr[v], f);
+        for (int i = 0; i < 8; ++i) {
+            lo = fminf(lo, f[i]);
+            hi = fmaxf(hi, f[i]);
+        }
+    }
+    return make_float2(lo, hi);
+}
+
+// Offset codes (q + z, or q + 8 when symmetric) of 16 packed bf16 pairs through
+// f = x * rcp and the rounding constant; dmax collects |f - rint(f)|.
+template <bool CLAMP>
+__device__ __forceinline__ void fast_codes(const uint32_t (&w)[16], float rcp, uint32_t coff, bool sym,
+                                           uint32_t (&word)[4], float& dmax) {
+    const float2 rcp2 = make_float2(rcp, rcp);
+    const float2 mag2 = make_float2(kRoundMagic, kRoundMagic);
+    const float2 nmag2 = make_float2(-kRoundMagic, -kRoundMagic);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+    float dm0 = 0.0f, dm1 = 0.0f;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t wv = w[4 * h + i];
+            const float2 x2 = make_float2(__uint_as_float(wv << 16), __uint_as_float(wv & 0xffff0000u));
+            const float2 f2 = __fmul2_rn(x2, rcp2);
+            const float2 t2 = __fadd2_rn(f2, mag2);
+            const float2 r2 = __fadd2_rn(t2, nmag2);    // rint(f), exact
+            const float2 d2 = __ffma2_rn(r2, neg1, f2);  // f - rint(f), exact
+            dm0 = fmaxf(dm0, fabsf(d2.x));
+            dm1 = fmaxf(dm1, fabsf(d2.y));
+            int c0 = (int)(__float_as_uint(t2.x) + coff), c1 = (int)(__float_as_uint(t2.y) + coff);
+            if (CLAMP) {  // offset codes: [0, 15] for both encodings
+                c0 = min(max(c0, 0), 15);
+                c1 = min(max(c1, 0), 15);
+            }
+            // elements 2i and 2i + 1 of the word: nibbles 2i and 2i + 1 (low first)
+            acc |= (uint32_t)c0 << (8 * i);
+            acc |= (uint32_t)c1 << (8 * i + 4);
+        }
+        word[h] = sym ? acc ^ 0x88888888u : acc;  // q + 8 -> two's-complement nibble
+    }
+    dmax = fmaxf(dm0, dm1);
+}
+
+__device__ __noinline__ uint32_t encode8_slow(const uint4 raw, const ScaleZero sz, bool symmetric) {
+    float v[8];
+    unpack_bf16x8(raw, v);
+    return encode8(v, sz, symmetric);
+}
+
+// g <= 256: each thread takes four consecutive segments (32 weights, four
+// 16-byte loads), so the per-group work is shared by 32 weights per thread;
+// L = g/32 lanes per group, 32/L groups per warp.
+//
+// Fast path (finite group, scale not saturated -- then |x/s| <= 15.01):
+//  - statistics with packed bf16x2 max/min that propagate NaN, so one test
+//    per thread tells whether its values are all non-NaN;
+//  - scale and zero without fp32 divisions (scale_zero_fast);
+//  - f = x * rcp(s) in packed fp32x2; t = f + 1.5*2^23 puts rint(f) (round
+//    half to even) in the low mantissa bits, so the code is bits(t) + const;
+//  - the quotient guard of rint_quotient: if some |f - rint(f)| is within
+//    2^-17 of 1/2, the thread redoes its codes with the IEEE division;
+//  - fl(x/s) and rint are monotone, so the codes of the group's extremes
+//    bound all its codes: when both are inside the code range (and neither
+//    is near a tie) no code needs clamping.
+// Anything else (NaN or Inf in the warp's groups, a saturated scale) takes
+// the general per-value path of encode8.
+constexpr int kUnitsPerThread = 2;  // 32-weight units in flight per thread
+
+// Fast code of x (offset form: q + z, or q + 8 when symmetric) and |f - rint(f)|.
+__device__ __forceinline__ int fast_code(float x, float rcp, uint32_t coff, float& dist) {
+    const float f = __fmul_rn(x, rcp);
+    const float t = __fadd_rn(f, kRoundMagic);
+    dist = fabsf(__fsub_rn(f, __fsub_rn(t, kRoundMagic)));
+    return (int)(__float_as_uint(t) + coff);
+}
 
 template <int L>
 __global__ void __launch_bounds__(kQuantThreads) quantize_small_group_kernel(
-    const uint4* __restrict__ W, int64_t nseg, int symmetric, uint32_t* __restrict__ qweight,
+    const uint4* __restrict__ W, int64_t nunit, int symmetric, uint32_t* __restrict__ qweight,
     uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros, uint32_t* status) {
     const int lane = threadIdx.x & 31;
+    const bool sym = symmetric != 0;
     bool nonfinite = false, range = false;
-    const int64_t stride = (int64_t)gridDim.x * (kQuantThreads * kSegPerThread);
-    for (int64_t base = (int64_t)blockIdx.x * (kQuantThreads * kSegPerThread) + threadIdx.x; base - threadIdx.x < nseg;
-         base += stride) {
-        uint4 raw[kSegPerThread];
+    const int64_t stride = (int64_t)gridDim.x * (kQuantThreads * kUnitsPerThread);
+    for (int64_t base = (int64_t)blockIdx.x * (kQuantThreads * kUnitsPerThread) + threadIdx.x;
+         base - threadIdx.x < nunit; base += stride) {
+        uint4 raw[kUnitsPerThread][4];
 #pragma unroll
-        for (int u = 0; u < kSegPerThread; ++u) {
-            const int64_t seg = base + (int64_t)u * kQuantThreads;
-            raw[u] = seg < nseg ? ld_nc_v4(W + seg) : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < kUnitsPerThread; ++u) {
+            const int64_t un = base + (int64_t)u * kQuantThreads;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) raw[u][v] = un < nunit ? ld_nc_v4(W + 4 * un + v) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int u = 0; u < kSegPerThread; ++u) {
-            const int64_t seg = base + (int64_t)u * kQuantThreads;
-            float v[8];
-            unpack_bf16x8(raw[u], v);
-            float lo = 0.0f, hi = 0.0f;
+        for (int u = 0; u < kUnitsPerThread; ++u) {
+            const int64_t un = base + (int64_t)u * kQuantThreads;
+            uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                nonfinite |= !isfinite(v[i]);
-                lo = fminf(lo, v[i]);
-                hi = fmaxf(hi, v[i]);
+            for (int v = 0; v < 4; ++v) {
+                w[4 * v] = raw[u][v].x;
+                w[4 * v + 1] = raw[u][v].y;
+                w[4 * v + 2] = raw[u][v].z;
+                w[4 * v + 3] = raw[u][v].w;
+            }
+            // ---- statistics of the thread's 32 values (NaN propagates) ----
+            __nv_bfloat162 mx = __hmax2_nan(bits_bf2(w[0]), bits_bf2(w[1]));
+            __nv_bfloat162 mn = __hmin2_nan(bits_bf2(w[0]), bits_bf2(w[1]));
+#pragma unroll
+            for (int i = 2; i < 16; ++i) {
+                mx = __hmax2_nan(mx, bits_bf2(w[i]));
+                mn = __hmin2_nan(mn, bits_bf2(w[i]));
+            }
+            const uint32_t mxb = bf2_bits(mx), mnb = bf2_bits(mn);
+            const float mx0 = __uint_as_float(mxb << 16), mx1 = __uint_as_float(mxb & 0xffff0000u);
+            const bool has_nan = isnan(mx0) || isnan(mx1);
+            float hi = fmaxf(fmaxf(mx0, mx1), 0.0f);
+            float lo = fminf(fminf(__uint_as_float(mnb << 16), __uint_as_float(mnb & 0xffff0000u)), 0.0f);
+            if (__any_sync(0xffffffffu, has_nan) && has_nan) {  // NaN inputs are skipped by the statistics
+                const float2 m = nan_skipping_min_max(raw[u][0], raw[u][1], raw[u][2], raw[u][3]);
+                lo = m.x;
+                hi = m.y;
             }
 #pragma unroll
             for (int o = 1; o < L; o <<= 1) {
                 lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
                 hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
             }
-            ScaleZero sz = scale_zero(lo, hi, symmetric != 0);
-            if (seg < nseg) {
-                range |= sz.range;
-                qweight[seg] = encode8(v, sz, symmetric != 0);
+            const bool inf = isinf(lo) || isinf(hi);
+            nonfinite |= has_nan || inf;
+            float rcp;
+            const ScaleZero sz = scale_zero_fast(lo, hi, sym, rcp);
+            if (un < nunit) range |= sz.range;
+            uint32_t word[4];
+            const bool general = __any_sync(0xffffffffu, has_nan || inf || sz.range);
+            bool slow = general;
+            if (!general) {
+                const uint32_t coff = (uint32_t)(sym ? 8 : sz.z) - kRoundMagicBits;
+                float dlo, dhi;
+                const int clo = fast_code(lo, rcp, coff, dlo), chi = fast_code(hi, rcp, coff, dhi);
+                const float tie = 0.5f - 0x1p-17f;
+                const bool clamp = __any_sync(0xffffffffu, clo < 0 || chi > 15 || dlo > tie || dhi > tie);
+                float dmax;
+                if (clamp)
+                    fast_codes<true>(w, rcp, coff, sym, word, dmax);
+                else
+                    fast_codes<false>(w, rcp, coff, sym, word, dmax);
+                slow = dmax > tie;
+            }
+            if (slow)
+                for (int h = 0; h < 4; ++h) word[h] = encode8_slow(raw[u][h], sz, sym);
+            if (un < nunit) {
+                reinterpret_cast<uint4*>(qweight)[un] = make_uint4(word[0], word[1], word[2], word[3]);
                 if ((lane & (L - 1)) == 0) {
-                    const int64_t gi = seg / L;
+                    const int64_t gi = un / L;
                     scales[gi] = sz.s16;
-                    if (!symmetric) zeros[gi] = __half_as_ushort(__int2half_rn(sz.z));
+                    if (!sym) zeros[gi] = __half_as_ushort(__int2half_rn(sz.z));
                 }
             }
         }
@@ -255,25 +428,25 @@ cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, i
     const int64_t P = d_out * d_in;
     const uint4* W4 = static_cast<const uint4*>(W);
     if (g <= 256) {
-        const int64_t nseg = P / 8;
-        const int64_t per_block = (int64_t)kQuantThreads * kSegPerThread;
-        int64_t blocks = (nseg + per_block - 1) / per_block;
+        const int64_t nunit = P / 32;
+        const int64_t per_block = (int64_t)kQuantThreads * kUnitsPerThread;
+        int64_t blocks = (nunit + per_block - 1) / per_block;
         if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
         switch (g) {
             case 32:
-                quantize_small_group_kernel<4><<<blocks, kQuantThreads, 0, stream>>>(W4, nseg, symmetric, qweight,
+                quantize_small_group_kernel<1><<<blocks, kQuantThreads, 0, stream>>>(W4, nunit, symmetric, qweight,
                                                                                        scales, zeros, status);
                 break;
             case 64:
-                quantize_small_group_kernel<8><<<blocks, kQuantThreads, 0, stream>>>(W4, nseg, symmetric, qweight,
+                quantize_small_group_kernel<2><<<blocks, kQuantThreads, 0, stream>>>(W4, nunit, symmetric, qweight,
                                                                                        scales, zeros, status);
                 break;
             case 128:
-                quantize_small_group_kernel<16><<<blocks, kQuantThreads, 0, stream>>>(W4, nseg, symmetric, qweight,
-                                                                                        scales, zeros, status);
+                quantize_small_group_kernel<4><<<blocks, kQuantThreads, 0, stream>>>(W4, nunit, symmetric, qweight,
+                                                                                       scales, zeros, status);
                 break;
             case 256:
-                quantize_small_group_kernel<32><<<blocks, kQuantThreads, 0, stream>>>(W4, nseg, symmetric, qweight,
+                quantize_small_group_kernel<8><<<blocks, kQuantThreads, 0, stream>>>(W4, nunit, symmetric, qweight,
                                                                                         scales, zeros, status);
                 break;
             default:

@@ -70,6 +70,22 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t shifted, const GroupCo
     return bf2_bits(w);
 }
 
+// Group constants packed in 8 bytes: (s_hi, s_lo) and (128 + z, xmask half),
+// each bf16 once; unpack_consts replicates them into the bf16x2 form.
+__device__ __forceinline__ GroupConsts unpack_consts(uint2 v) {
+    GroupConsts c;
+    c.s_hi = __byte_perm(v.x, v.x, 0x1010);
+    c.s_lo = __byte_perm(v.x, v.x, 0x3232);
+    c.zm = __byte_perm(v.y, v.y, 0x1010);
+    c.xmask = __byte_perm(v.y, v.y, 0x3232);
+    return c;
+}
+
+__device__ __forceinline__ uint2 pack_consts(uint16_t s16, int z, bool sym) {
+    const GroupConsts g = make_group_consts(s16, z, sym);
+    return make_uint2((g.s_hi & 0xffffu) | (g.s_lo << 16), (g.zm & 0xffffu) | (g.xmask << 16));
+}
+
 // Dequantize one packed word (8 nibbles, low nibble first).
 // out[p] = (x_hat(nibble p), x_hat(nibble p + 4)) for p = 0..3.
 __device__ __forceinline__ void dequant_word_pairs(uint32_t w, const GroupConsts& c, uint32_t out[4]) {
@@ -147,6 +163,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of an mbarrier phase (no suspend).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -211,6 +240,22 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait_prior() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Hardware named barriers (ids 1..15; id 0 is __syncthreads).  bar.arrive
+// counts the calling warp and continues; bar.sync counts it and waits until
+// `nthreads` threads have arrived.
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ uint16_t ld_nc_u16(const uint16_t* p) {
+    uint16_t r;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
 }
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {

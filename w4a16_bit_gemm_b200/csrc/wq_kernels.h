@@ -45,6 +45,15 @@ struct LaunchOptions {
 cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_sms, const LaunchOptions& opt,
                         cudaStream_t stream);
 
+// M <= 2 on tensor cores (dequantized weights as the A operand in tensor
+// memory); cudaErrorNotSupported for shapes it does not take.
+cudaError_t launch_gemv_tc(const uint32_t* qweight, const GemvArgs& a, int num_sms, const LaunchOptions& opt,
+                           cudaStream_t stream);
+
+// WQ_GEMV_TC=0 in the environment keeps M <= 2 off the tensor-memory kernel
+// (read once per process).
+bool gemv_tc_disabled();
+
 // Prefill GEMM on tcgen05 tensor cores, any M (used for M > 16).
 struct GemmArgs {
     const void* X;           // bf16 [M][K]
