@@ -385,28 +385,28 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 }
 
 // ------------------------------------------------------------------------
-// M = 1: CUDA-core dot product.  The m16n8k16 MMA would waste 7/8 of its
-// n dimension on one token, so the single-token GEMV multiplies on the FMA
-// pipe instead: fma.rn.f32.bf16 takes the exact bf16 x_hat and the bf16
-// activation as operands and accumulates in fp32 (one rounding per product
-// and accumulation, as an fp32 FFMA of the widened values).
+// M = 1: dequant on the CUDA cores, products and sums on the tensor pipe
+// (fp32 accumulation).  One token fills 1/8 of the m16n8k16 n dimension, but
+// the MMA still replaces the per-weight multiply-add and register splitting
+// the CUDA cores would otherwise spend on every weight.
 // - A CTA's rows are one contiguous byte range of qweight, so the producer
 //   moves them with 1D bulk copies of <= 16 KB (the copy engine streams these
 //   at HBM rate; many small row pieces it cannot).  A chunk is RC consecutive
 //   rows; chunks are resident when they fit, else they cycle through a ring
 //   where every consumer warp consumes every chunk in order.
-// - A unit is (row, 1024-k part): lane l takes the 32-k slice l of the part
-//   (4 packed words, one LDS.128; a warp reads 512 contiguous bytes).  Units
-//   are dealt round-robin to 16 consumer warps, so rows need no padding; a
-//   warp keeps its activation slice (fp32) in registers while its part
-//   repeats.
-// - Each unit's 32 lane partials are folded to 8 with two shuffles and
-//   parked in shared memory; a fixed-order sum per row finishes (deterministic).
+// - Products on the tensor pipe with mma.sync m16n8k16: a unit is (16-row
+//   block, 128-k step).  Lane (g, t) = (lane / 4, lane % 4) dequantizes the
+//   32-k slice 4 * step + t of rows g and g + 8 (one 16-byte word load per
+//   row); its bf16x2 pairs (nibble p, nibble p + 4) are A-fragment registers
+//   directly, and the staged activation pairs are the matching B fragments
+//   (all 8 columns of B carry the same token, so any column of D is y).
+//   Steps are dealt round-robin to 16 consumer warps; each warp parks its
+//   per-row partial, and a fixed-order sum per row finishes (deterministic).
 // ------------------------------------------------------------------------
 
 constexpr int kM1Warps = 16;
 constexpr int kM1Threads = (kM1Warps + 1) * 32;
-constexpr int kM1PartK = 1024;            // k per unit (32 lanes x 32 k)
+constexpr int kM1StepK = 128;             // k per unit (4 lanes x 32 k)
 constexpr int kM1SmemBudget = 200 * 1024;
 constexpr int kM1MaxSlots = 16;
 constexpr int kM1CopyPiece = 16384;
@@ -416,29 +416,17 @@ struct GemvM1Layout {
 };
 
 // cst: 16 B per (row, group); xs: 64 B per 32-k slice (activation pairs
-// matching the nibble pairs); red: [rows][parts][8] floats.
+// matching the nibble pairs); red: [rows][consumer warps] floats.
 __host__ __device__ inline GemvM1Layout gemv_m1_layout(const GemvArgs& a) {
     GemvM1Layout L;
     const int nsl = (a.K + 31) / 32;
-    const int nkp = (a.K + kM1PartK - 1) / kM1PartK;
     L.bar_off = 0;
     L.cst_off = round_up(16 * a.nslots, 128);
     L.xs_off = L.cst_off + round_up(a.BR * a.G * 16, 128);
     L.red_off = L.xs_off + round_up(nsl * 64, 128);
-    L.slot_off = round_up(L.red_off + a.BR * nkp * 8 * 4, 1024);
+    L.slot_off = round_up(L.red_off + a.BR * kM1Warps * 4, 1024);
     L.total = L.slot_off + a.nslots * a.slot_bytes + 1024;
     return L;
-}
-
-// acc0 += lo(w2) * lo(x2), acc1 += hi(w2) * hi(x2), each rounded once into fp32.
-__device__ __forceinline__ void fma2_bf16_f32(float& acc0, float& acc1, uint32_t w2, uint32_t x2) {
-    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
-        "mov.b32 {wl, wh}, %2;\n\t"
-        "mov.b32 {xl, xh}, %3;\n\t"
-        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
-        "fma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
-        : "+f"(acc0), "+f"(acc1)
-        : "r"(w2), "r"(x2));
 }
 
 __global__ void __launch_bounds__(kM1Threads, 1)
@@ -461,7 +449,7 @@ __global__ void __launch_bounds__(kM1Threads, 1)
     const int nch = (nrows + RC - 1) / RC;
     const int64_t row_bytes = (int64_t)a.K / 2;
     const int nsl = (a.K + 31) / 32;
-    const int nkp = (a.K + kM1PartK - 1) / kM1PartK;
+    const int nks = (a.K + kM1StepK - 1) / kM1StepK;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.nslots; ++i) {
@@ -570,8 +558,10 @@ __global__ void __launch_bounds__(kM1Threads, 1)
     }
     named_sync(1, nthreads_c);
 
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const GroupConsts zero_consts = {0u, 0u, 0u, 0u};  // x_hat = 0 for rows past the chunk
     uint32_t xr[16];
-    int cached_kp = -1;
+    int cached_ks = -1;
     for (int c = 0; c < nch; ++c) {
         const int slot = c % a.nslots;
         const bool landed = mbar_wait(&full[slot], (uint32_t)(c / a.nslots) & 1u, a.status);
@@ -581,57 +571,58 @@ __global__ void __launch_bounds__(kM1Threads, 1)
         }
         const uint8_t* sp = slots + (size_t)slot * a.slot_bytes;
         const int rows = min(RC, nrows - c * RC);
-        // units u = rl * nkp + kp dealt round-robin; (rl, kp) advanced without division
-        int rl = warp / nkp, kp = warp - (warp / nkp) * nkp;
-        const int drl = kM1Warps / nkp, dkp = kM1Warps - drl * nkp;
-        for (int u = warp; u < rows * nkp; u += kM1Warps) {
-            const int r = c * RC + rl;  // CTA row
-            const int s = kp * 32 + lane;
-            float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-            if (s < nsl) {
-                const int k0 = s * 32;
-                if (kp != cached_kp) {  // the activation slice stays in registers while kp repeats
+        for (int rb = 0; rb * 16 < rows; ++rb) {
+            const int ra = rb * 16 + g8, rbb = ra + 8;  // chunk rows of this lane
+            const bool va = ra < rows, vb = rbb < rows;
+            float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int ks = warp; ks < nks; ks += kM1Warps) {
+                const int s = ks * 4 + t4;  // the lane's 32-k slice
+                const bool vs = s < nsl;
+                if (ks != cached_ks) {  // activation pairs of the slice: the B fragments
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4 v = xs[s * 4 + q];
+                        const uint4 v = vs ? xs[s * 4 + q] : make_uint4(0, 0, 0, 0);
                         xr[4 * q] = v.x; xr[4 * q + 1] = v.y; xr[4 * q + 2] = v.z; xr[4 * q + 3] = v.w;
                     }
-                    cached_kp = kp;
+                    cached_ks = ks;
                 }
-                const uint4 w = *reinterpret_cast<const uint4*>(sp + rl * row_bytes + s * 16);
-                const uint4 kc = cst[r * a.G + (a.g_shift >= 0 ? (k0 >> a.g_shift) : k0 / a.g)];
-                const GroupConsts gc = {kc.x, kc.y, kc.z, kc.w};
-                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                const int gi = a.g_shift >= 0 ? ((s * 32) >> a.g_shift) : (s * 32) / a.g;
+                uint4 wa = make_uint4(0, 0, 0, 0), wb = wa;
+                GroupConsts ka = zero_consts, kb = zero_consts;
+                if (va && vs) {
+                    wa = *reinterpret_cast<const uint4*>(sp + ra * row_bytes + s * 16);
+                    const uint4 k4 = cst[(c * RC + ra) * a.G + gi];
+                    ka = {k4.x, k4.y, k4.z, k4.w};
+                }
+                if (vb && vs) {
+                    wb = *reinterpret_cast<const uint4*>(sp + rbb * row_bytes + s * 16);
+                    const uint4 k4 = cst[(c * RC + rbb) * a.G + gi];
+                    kb = {k4.x, k4.y, k4.z, k4.w};
+                }
+                const uint32_t wva[4] = {wa.x, wa.y, wa.z, wa.w}, wvb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    uint32_t pr[4];
-                    dequant_word_pairs(wv[j], gc, pr);
-                    fma2_bf16_f32(a0, a1, pr[0], xr[4 * j + 0]);
-                    fma2_bf16_f32(a2, a3, pr[1], xr[4 * j + 1]);
-                    fma2_bf16_f32(a0, a1, pr[2], xr[4 * j + 2]);
-                    fma2_bf16_f32(a2, a3, pr[3], xr[4 * j + 3]);
+                    uint32_t pa[4], pb[4];
+                    dequant_word_pairs(wva[j], ka, pa);
+                    dequant_word_pairs(wvb[j], kb, pb);
+                    mma_16816(d, pa[0], pb[0], pa[1], pb[1], xr[4 * j + 0], xr[4 * j + 1]);
+                    mma_16816(d, pa[2], pb[2], pa[3], pb[3], xr[4 * j + 2], xr[4 * j + 3]);
                 }
             }
-            float v = (a0 + a1) + (a2 + a3);
-            v += __shfl_xor_sync(0xffffffffu, v, 16);
-            v += __shfl_xor_sync(0xffffffffu, v, 8);
-            if (lane < 8) red[(r * nkp + kp) * 8 + lane] = v;
-            rl += drl;
-            kp += dkp;
-            if (kp >= nkp) {
-                kp -= nkp;
-                ++rl;
+            // d = (D[ra][2t], D[ra][2t+1], D[rb][2t], D[rb][2t+1]); every column holds the token
+            if (t4 == 0) {
+                if (va) red[(c * RC + ra) * kM1Warps + warp] = d[0];
+                if (vb) red[(c * RC + rbb) * kM1Warps + warp] = d[2];
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
     }
     named_sync(1, nthreads_c);
-    // each row's parked partials summed by one warp: lane-strided partial sums,
-    // then a shuffle tree (a fixed order, so the result is deterministic)
+    // each row's parked partials (one per consumer warp) summed by one warp in a
+    // fixed order (a shuffle tree), so the result is deterministic
     for (int r = warp; r < nrows; r += kM1Warps) {
-        float v = 0.0f;
-        for (int q = lane; q < nkp * 8; q += 32) v += red[r * nkp * 8 + q];
+        float v = lane < kM1Warps ? red[r * kM1Warps + lane] : 0.0f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if (lane == 0 && !abort_flag) {
