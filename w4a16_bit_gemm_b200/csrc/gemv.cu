@@ -461,6 +461,10 @@ __global__ void __launch_bounds__(kM1Threads, 1)
     }
     __syncthreads();
 
+    // the next launch may start as soon as SM resources allow: it only streams
+    // weights and scales before its own griddepcontrol.wait
+    pdl_launch_dependents();
+
     if (warp == kM1Warps) {
         // ---------------- producer: contiguous bulk copies ----------------
         if (lane == 0) {
@@ -484,7 +488,6 @@ __global__ void __launch_bounds__(kM1Threads, 1)
             }
         }
         __syncwarp();
-        pdl_launch_dependents();
         return;
     }
 
