@@ -111,6 +111,15 @@ def _load(path: str | None = None):
             lib.wqo_bf16_to_f32.restype = ctypes.c_float
             lib.wqo_dequant_one.argtypes = [ctypes.c_uint16, ctypes.c_int32, ctypes.c_int32]
             lib.wqo_dequant_one.restype = ctypes.c_uint16
+            lib.wqo_quantize_clip.argtypes = [P, i64, i64, i64, i32, i32, P, P, P, P, P, i32]
+            lib.wqo_quantize_clip.restype = i32
+            lib.wqo_quantize_group_range.argtypes = [P, i64, i32, i32, ctypes.c_float, ctypes.c_float,
+                                                     ctypes.c_float, P, P, P]
+            lib.wqo_quantize_group_range.restype = ctypes.c_uint32
+            lib.wqo_group_sq_error.argtypes = [P, i64, P, ctypes.c_uint16, ctypes.c_int32]
+            lib.wqo_group_sq_error.restype = ctypes.c_double
+            lib.wqo_clip_alpha.argtypes = [i32]
+            lib.wqo_clip_alpha.restype = ctypes.c_float
             for nm in ("wqo_f32_to_f16_array", "wqo_f32_to_bf16_array", "wqo_f16_to_f32_array"):
                 getattr(lib, nm).argtypes = [P, i64, P]
                 getattr(lib, nm).restype = None
@@ -198,6 +207,65 @@ def quantize(W_bits: np.ndarray, group_size: int, bits: int = 4, symmetric: bool
     if rc != 0:
         raise ValueError("oracle quantize rejected its arguments")
     return codes, scales, zeros, int(flags.value)
+
+
+CLIP_CANDIDATES = 11
+
+
+def quantize_clip(W_bits: np.ndarray, group_size: int, symmetric: bool = False, bits: int = 4,
+                  nthreads: int | None = None):
+    """Group-wise quantization with the MSE-optimal clipping search
+    ([P1 Clipping Trade-off]; [P2 calibration 4, MSE-optimal]).
+
+    Returns ``(codes, scales, zeros or None, flags, best)`` with ``best`` the
+    chosen candidate index per group (uint8 [d_out, G]; alpha = clip_alpha(i)).
+    """
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    d_out, d_in = W_bits.shape
+    G = d_in // group_size
+    codes = np.empty((d_out, d_in), np.int32)
+    scales = np.empty((d_out, G), np.uint16)
+    zeros = None if symmetric else np.empty((d_out, G), np.uint16)
+    best = np.empty((d_out, G), np.uint8)
+    flags = ctypes.c_uint32(0)
+    rc = _load().wqo_quantize_clip(_ptr(W_bits), d_out, d_in, group_size, bits, int(symmetric), _ptr(codes),
+                                   _ptr(scales), _ptr(zeros) if zeros is not None else None, _ptr(best),
+                                   ctypes.cast(ctypes.pointer(flags), ctypes.c_void_p),
+                                   nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle clip quantize rejected its arguments")
+    return codes, scales, zeros, int(flags.value), best
+
+
+def quantize_clip_pack4(W_bits: np.ndarray, group_size: int = 128, symmetric: bool = False,
+                        nthreads: int | None = None):
+    """quantize_clip + pack4: (qweight, scales, zeros, flags, codes, best)."""
+    codes, scales, zeros, flags, best = quantize_clip(W_bits, group_size, symmetric, nthreads=nthreads)
+    return pack4(codes), scales, zeros, flags, codes, best
+
+
+def clip_alpha(i: int) -> float:
+    return float(_load().wqo_clip_alpha(int(i)))
+
+
+def quantize_group_range(x_bits: np.ndarray, lo: float, hi: float, amax: float, symmetric: bool = False,
+                         bits: int = 4):
+    """One group quantized on a given range: (codes int32, s16, z, flags)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    codes = np.empty(x_bits.shape[0], np.int32)
+    s16 = ctypes.c_uint16(0)
+    z = ctypes.c_int32(0)
+    f = _load().wqo_quantize_group_range(_ptr(x_bits), x_bits.shape[0], bits, int(symmetric), lo, hi, amax,
+                                         _ptr(codes), ctypes.cast(ctypes.pointer(s16), ctypes.c_void_p),
+                                         ctypes.cast(ctypes.pointer(z), ctypes.c_void_p))
+    return codes, int(s16.value), int(z.value), int(f)
+
+
+def group_sq_error(x_bits: np.ndarray, codes: np.ndarray, s16: int, z: int) -> float:
+    """The oracle's fp64 squared reconstruction error of one group."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    codes = np.ascontiguousarray(codes, dtype=np.int32)
+    return float(_load().wqo_group_sq_error(_ptr(x_bits), x_bits.shape[0], _ptr(codes), s16, z))
 
 
 def pack4(codes: np.ndarray) -> np.ndarray:

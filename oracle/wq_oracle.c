@@ -178,29 +178,15 @@ static int clamp_to_int(float v, int lo, int hi) {
     return (int)v;
 }
 
-/* One group: derive (s, z) and the codes of g consecutive weights of one row.
- * x: g bf16 words; codes: g ints; returns flags. */
-static uint32_t quantize_group(const uint16_t* x, int64_t g, const wqo_qparams* p,
-                               int32_t* codes, uint16_t* s_out, uint16_t* z_out) {
+/* Scale and zero point of a group whose range is [lo, hi] (asymmetric, lo <= 0
+ * <= hi) or [-amax, amax] (symmetric); then the codes of its g weights.
+ * Returns WQO_FLAG_RANGE if the fp16 scale saturated. */
+static uint32_t quantize_with_range(const uint16_t* x, int64_t g, const wqo_qparams* p, float lo,
+                                    float hi, float amax, int32_t* codes, uint16_t* s_out,
+                                    int* z_out) {
     int qmin, qmax;
     code_range(p, &qmin, &qmax);
     uint32_t flags = 0;
-
-    /* statistics [P1 Symmetric / Asymmetric]; range widened to contain 0 */
-    float lo = 0.0f, hi = 0.0f, amax = 0.0f;
-#if WQO_MUTANT == 4 /* mistake: range not widened to contain zero */
-    lo = INFINITY;
-    hi = -INFINITY;
-#endif
-    for (int64_t k = 0; k < g; ++k) {
-        float v = wqo_bf16_to_f32(x[k]);
-        if (!isfinite(v)) flags |= WQO_FLAG_NONFINITE;
-        if (isnan(v)) continue;
-        if (v < lo) lo = v;
-        if (v > hi) hi = v;
-        float av = fabsf(v);
-        if (av > amax) amax = av;
-    }
 
     /* scale in fp32, stored as fp16 */
     float s32;
@@ -248,6 +234,34 @@ static uint32_t quantize_group(const uint16_t* x, int64_t g, const wqo_qparams* 
         codes[k] = clamp_to_int(t + (float)z, qmin, qmax);
     }
     *s_out = s16;
+    *z_out = z;
+    return flags;
+}
+
+/* One group: derive (s, z) and the codes of g consecutive weights of one row.
+ * x: g bf16 words; codes: g ints; returns flags. */
+static uint32_t quantize_group(const uint16_t* x, int64_t g, const wqo_qparams* p,
+                               int32_t* codes, uint16_t* s_out, uint16_t* z_out) {
+    uint32_t flags = 0;
+
+    /* statistics [P1 Symmetric / Asymmetric]; range widened to contain 0 */
+    float lo = 0.0f, hi = 0.0f, amax = 0.0f;
+#if WQO_MUTANT == 4 /* mistake: range not widened to contain zero */
+    lo = INFINITY;
+    hi = -INFINITY;
+#endif
+    for (int64_t k = 0; k < g; ++k) {
+        float v = wqo_bf16_to_f32(x[k]);
+        if (!isfinite(v)) flags |= WQO_FLAG_NONFINITE;
+        if (isnan(v)) continue;
+        if (v < lo) lo = v;
+        if (v > hi) hi = v;
+        float av = fabsf(v);
+        if (av > amax) amax = av;
+    }
+
+    int z;
+    flags |= quantize_with_range(x, g, p, lo, hi, amax, codes, s_out, &z);
     if (z_out) *z_out = wqo_f32_to_f16((float)z);
     return flags;
 }
@@ -332,6 +346,149 @@ int wqo_quantize(const uint16_t* W, int64_t d_out, int64_t d_in, int64_t g, int 
     if (!symmetric && !zeros) return -1;
     quant_ctx c = {W, d_in, g, {bits, symmetric, narrow}, codes, scales, symmetric ? NULL : zeros};
     uint32_t f = run_rows(quant_rows, &c, d_out, nthreads);
+    if (flags) *flags = f;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MSE-optimal clipping per group                                            */
+/* [P1 Clipping Trade-off]: a range set by one large value coarsens every    */
+/* level; clipping it trades that value's error for the rest's.  The         */
+/* threshold is chosen to minimise the local reconstruction error            */
+/* [P2 calibration section 4: MSE-optimal, argmin ||x - x_dq||^2, chosen per  */
+/* channel/group independently].                                             */
+/* Readings (the pages give no grid or summation order):                     */
+/*  - candidates shrink the RTN range by alpha_i = fl32((20 - i) / 20),      */
+/*    i = 0..10 (1.00, 0.95, ..., 0.50): lo_i = fl32(alpha_i lo),             */
+/*    hi_i = fl32(alpha_i hi) (amax_i likewise); scale, zero and codes follow */
+/*    the RTN formulas on that range, values outside it are clamped by the    */
+/*    code range;                                                            */
+/*  - the error is sum_k (x_k - x_hat_k)^2 over the finite x_k, x_hat_k the   */
+/*    bf16 dequantized value; differences and squares are exact in fp64; the */
+/*    sum runs over runs of 8 consecutive weights in order, then a pairwise  */
+/*    tree over the runs in index order (g/8 must be a power of two);         */
+/*  - the smallest error wins; ties go to the smaller i (less clipping).      */
+/* alpha_0 = 1 is plain RTN, so the chosen error never exceeds RTN's.        */
+/* ------------------------------------------------------------------------ */
+
+#define WQO_CLIP_CANDIDATES 11
+
+uint16_t wqo_dequant_one(uint16_t s16, int32_t q, int32_t z);
+
+/* One group quantized on a given range (test access to the candidate step). */
+uint32_t wqo_quantize_group_range(const uint16_t* x, int64_t g, int bits, int symmetric, float lo,
+                                  float hi, float amax, int32_t* codes, uint16_t* s16, int32_t* z) {
+    wqo_qparams p = {bits, symmetric, 0};
+    int zi;
+    uint32_t f = quantize_with_range(x, g, &p, lo, hi, amax, codes, s16, &zi);
+    *z = zi;
+    return f;
+}
+
+float wqo_clip_alpha(int i) { return (float)(20 - i) / 20.0f; }
+
+/* Squared reconstruction error of one group in the order stated above. */
+double wqo_group_sq_error(const uint16_t* x, int64_t g, const int32_t* codes, uint16_t s16, int z) {
+    int64_t runs = g / 8;
+    double part[512];
+    for (int64_t r = 0; r < runs; ++r) {
+        double acc = 0.0;
+        for (int64_t k = 8 * r; k < 8 * r + 8; ++k) {
+            float v = wqo_bf16_to_f32(x[k]);
+            if (!isfinite(v)) continue;
+            double xh = (double)wqo_bf16_to_f32(wqo_dequant_one(s16, codes[k], z));
+#if WQO_MUTANT == 9 /* mistake: absolute error instead of its square */
+            double e = fabs((double)v - xh);
+#else
+            double e = ((double)v - xh) * ((double)v - xh);
+#endif
+            acc += e;
+        }
+        part[r] = acc;
+    }
+    for (int64_t w = 1; w < runs; w *= 2)
+        for (int64_t r = 0; r + w < runs; r += 2 * w) part[r] = part[r] + part[r + w];
+    return part[0];
+}
+
+/* One group with the clipping search; *best gets the chosen candidate index. */
+static uint32_t quantize_group_clip(const uint16_t* x, int64_t g, const wqo_qparams* p,
+                                    int32_t* codes, uint16_t* s_out, uint16_t* z_out,
+                                    uint8_t* best) {
+    uint32_t flags = 0;
+    float lo = 0.0f, hi = 0.0f, amax = 0.0f;
+    for (int64_t k = 0; k < g; ++k) {
+        float v = wqo_bf16_to_f32(x[k]);
+        if (!isfinite(v)) flags |= WQO_FLAG_NONFINITE;
+        if (isnan(v)) continue;
+        if (v < lo) lo = v;
+        if (v > hi) hi = v;
+        float av = fabsf(v);
+        if (av > amax) amax = av;
+    }
+    int32_t cand[1024];
+    double best_err = 0.0;
+    int best_i = -1, best_z = 0;
+    uint16_t best_s = 0;
+    uint32_t best_flags = 0;
+    for (int i = 0; i < WQO_CLIP_CANDIDATES; ++i) {
+        float a = wqo_clip_alpha(i);
+        uint16_t s16;
+        int z;
+        uint32_t f = quantize_with_range(x, g, p, a * lo, a * hi, a * amax, cand, &s16, &z);
+        double err = wqo_group_sq_error(x, g, cand, s16, z);
+#if WQO_MUTANT == 10 /* mistake: the largest error wins */
+        if (best_i < 0 || err > best_err) {
+#else
+        if (best_i < 0 || err < best_err) {
+#endif
+            best_i = i;
+            best_err = err;
+            best_s = s16;
+            best_z = z;
+            best_flags = f;
+            for (int64_t k = 0; k < g; ++k) codes[k] = cand[k];
+        }
+    }
+    *s_out = best_s;
+    if (z_out) *z_out = wqo_f32_to_f16((float)best_z);
+    if (best) *best = (uint8_t)best_i;
+    return flags | best_flags;
+}
+
+typedef struct {
+    const uint16_t* W;
+    int64_t d_in, g;
+    wqo_qparams p;
+    int32_t* codes;
+    uint16_t* scales;
+    uint16_t* zeros;
+    uint8_t* best;
+} clip_ctx;
+
+static void clip_rows(void* vctx, int64_t r0, int64_t r1, uint32_t* flags) {
+    clip_ctx* c = (clip_ctx*)vctx;
+    int64_t ng = c->d_in / c->g;
+    for (int64_t r = r0; r < r1; ++r)
+        for (int64_t j = 0; j < ng; ++j) {
+            int64_t off = r * c->d_in + j * c->g;
+            *flags |= quantize_group_clip(c->W + off, c->g, &c->p, c->codes + off, c->scales + r * ng + j,
+                                          c->zeros ? c->zeros + r * ng + j : NULL,
+                                          c->best ? c->best + r * ng + j : NULL);
+        }
+}
+
+/* As wqo_quantize, with the clipping search; best: chosen candidate index per
+ * group [d_out][d_in/g] (may be NULL).  g/8 must be a power of two, g <= 1024. */
+int wqo_quantize_clip(const uint16_t* W, int64_t d_out, int64_t d_in, int64_t g, int bits,
+                      int symmetric, int32_t* codes, uint16_t* scales, uint16_t* zeros,
+                      uint8_t* best, uint32_t* flags, int nthreads) {
+    if (!W || !codes || !scales || d_out < 0 || d_in <= 0 || g < 8 || g > 1024 || d_in % g != 0) return -1;
+    if ((g % 8) != 0 || ((g / 8) & (g / 8 - 1)) != 0) return -1;
+    if (bits < 2 || bits > 8) return -1;
+    if (!symmetric && !zeros) return -1;
+    clip_ctx c = {W, d_in, g, {bits, symmetric, 0}, codes, scales, symmetric ? NULL : zeros, best};
+    uint32_t f = run_rows(clip_rows, &c, d_out, nthreads);
     if (flags) *flags = f;
     return 0;
 }

@@ -1,10 +1,12 @@
 """Planted mistakes: each mutant of the oracle (one plausible error compiled
 in with -DWQO_MUTANT=k) must fail at least one pin, and the real oracle must
 pass the same pins.  This shows the pins constrain every step: statistics,
-scale, zero point, rounding, packing, dequantization and the linear layer."""
+scale, zero point, rounding, packing, dequantization, the linear layer and
+the clipping search (error formula and selection)."""
 import pytest
 
 import oracle
+from tests import test_oracle_clip_pins as clip_pins
 from tests import test_oracle_pins as pins
 
 PINS = [
@@ -17,6 +19,9 @@ PINS = [
     pins.test_pack_layout_low_nibble_first,
     pins.test_dequant_exhaustive_against_library_rounding,
     pins.test_linear_special_cases_and_matmul,
+    clip_pins.test_error_formula_is_the_exact_sum_of_squares,
+    clip_pins.test_choice_is_the_exact_argmin,
+    clip_pins.test_never_worse_than_rtn,
 ]
 
 MUTANTS = {
@@ -27,6 +32,8 @@ MUTANTS = {
     5: "transposed weight in linear",
     6: "zero point dropped in dequant",
     7: "high nibble first",
+    9: "clip search sums absolute errors",
+    10: "clip search keeps the largest error",
 }
 
 
