@@ -312,6 +312,21 @@ def run_ours(args, dist: Dist):
     qb = quant_bytes(D, D, False)
     secondary["quantize"] = {"shape": "4096x4096", "GBps": qb / tq / 1e9, "us_per_launch": tq * 1e6,
                              "bytes_per_launch": qb, "frac_of_measured_hbm": qb / tq / 1e9 / hbm}
+    # quantization with the per-group MSE-optimal clipping search: throughput and
+    # the squared reconstruction error relative to RTN on the same weights
+    def qcfn():
+        for i in range(QC):
+            b.quantize_clip_mse(Ws[i], G128, False, out=qpacks[i])
+    gqc = capture(qcfn)
+    tqc = dist.max(timed_graph(gqc, max(3, qsteps // 4), 3, dist)) / (max(3, qsteps // 4) * QC)
+    p_clip = b.quantize_clip_mse(W, G128, False)
+    Wd = W.double()
+    err_clip = float(((Wd - b.dequantize(p_clip).double()) ** 2).sum())
+    err_rtn = float(((Wd - b.dequantize(p0).double()) ** 2).sum())
+    secondary["quantize_clip_mse"] = {"shape": "4096x4096", "GBps": qb / tqc / 1e9, "us_per_launch": tqc * 1e6,
+                                      "frac_of_measured_hbm": qb / tqc / 1e9 / hbm,
+                                      "sq_error_vs_rtn": err_clip / err_rtn}
+    del gqc, p_clip, Wd
     What = [torch.empty(D, D, dtype=torch.bfloat16, device="cuda") for _ in range(QC)]
 
     def dfn():

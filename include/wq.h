@@ -119,6 +119,35 @@ wq_status wq_quantize_rtn(const void* W_bf16, int64_t d_out, int64_t d_in, int32
                           void* zeros_fp16, void* stream);
 
 /*
+ * wq_quantize_clip_mse -- group-wise quantization with a per-group clipping
+ * search that minimises the reconstruction error ("Clipping Trade-off" of the
+ * first page cited above: a range set by one large value coarsens every
+ * level, so the threshold is chosen to minimise the local reconstruction
+ * error; the "Quantization Algorithms" notes, calibration section 4:
+ * MSE-optimal argmin ||x - x_dq||^2, independent per group).
+ *
+ * Candidate i = 0..10 shrinks the group's RTN range by alpha_i =
+ * fl32((20 - i) / 20) (1.00, 0.95, ..., 0.50); its scale, zero point and
+ * codes follow wq_quantize_rtn on that range (values outside it clamp to the
+ * end codes).  Its error is sum_k (x_k - x_hat_k)^2 over the group's finite
+ * x_k, with x_hat_k = bf16_rn(s (q_k - z)), computed in fp64 (difference,
+ * square rounded once, add; no fused multiply-add) sequentially over each run
+ * of 8 consecutive weights and then by a pairwise tree over the runs in
+ * index order.  The candidate with the smallest error is kept (ties: the
+ * smaller i); alpha_0 = 1 is plain RTN, so the error never exceeds RTN's.
+ *
+ * Arguments, layout and ownership as in wq_quantize_rtn; the output artifact
+ * has the same format, so wq_dequantize and wq_linear_w4a16 consume it as is.
+ * Errors: as wq_quantize_rtn; WQ_ERR_UNSUPPORTED for a group size other than
+ * 32, 64, 128 or 256.
+ * Device flags: WQ_DEVFLAG_NONFINITE; WQ_DEVFLAG_RANGE if the kept
+ * candidate's scale saturated.
+ */
+wq_status wq_quantize_clip_mse(const void* W_bf16, int64_t d_out, int64_t d_in, int32_t group_size,
+                               int32_t symmetric, uint32_t* qweight, void* scales_fp16,
+                               void* zeros_fp16, void* stream);
+
+/*
  * wq_dequantize -- x_hat = bf16_rn(s (q - z)) for every weight ("Affine
  * Quantization"; the "full dequantize then matmul" path B of the "Fused
  * low-bit kernel" section).  Arguments as in wq_quantize_rtn, with the packed

@@ -364,9 +364,10 @@ int wqo_quantize(const uint16_t* W, int64_t d_out, int64_t d_in, int64_t g, int 
 /*    the RTN formulas on that range, values outside it are clamped by the    */
 /*    code range;                                                            */
 /*  - the error is sum_k (x_k - x_hat_k)^2 over the finite x_k, x_hat_k the   */
-/*    bf16 dequantized value; differences and squares are exact in fp64; the */
-/*    sum runs over runs of 8 consecutive weights in order, then a pairwise  */
-/*    tree over the runs in index order (g/8 must be a power of two);         */
+/*    bf16 dequantized value, in fp64: the difference, its square rounded     */
+/*    once, then the add (no fused multiply-add); the sum runs over runs of 8  */
+/*    consecutive weights in order, then a pairwise tree over the runs in     */
+/*    index order (g/8 must be a power of two);                               */
 /*  - the smallest error wins; ties go to the smaller i (less clipping).      */
 /* alpha_0 = 1 is plain RTN, so the chosen error never exceeds RTN's.        */
 /* ------------------------------------------------------------------------ */

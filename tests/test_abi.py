@@ -27,7 +27,7 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for n in ("wq_quantize_rtn", "wq_dequantize", "wq_linear_w4a16", "wq_linear_workspace_bytes",
+    for n in ("wq_quantize_rtn", "wq_quantize_clip_mse", "wq_dequantize", "wq_linear_w4a16", "wq_linear_workspace_bytes",
               "wq_get_device_error", "wq_status_string", "wq_abi_version"):
         assert n in names
 
@@ -85,3 +85,19 @@ def test_dequantize_rejects(lib):
 
 def test_workspace_query(lib):
     assert lib.wq_linear_workspace_bytes(1, 4096, 4096) >= 0
+
+
+@pytest.mark.parametrize("case", [
+    dict(W=None), dict(W=FAKE + 8), dict(q=None), dict(d_in=1000, g=128), dict(zeros=None), dict(sym=1),
+])
+def test_quantize_clip_rejects(lib, case):
+    a = dict(W=FAKE, d_out=4, d_in=256, g=128, sym=0, q=FAKE, s=FAKE, zeros=FAKE)
+    a.update(case)
+    st = lib.wq_quantize_clip_mse(a["W"], a["d_out"], a["d_in"], a["g"], a["sym"], a["q"], a["s"], a["zeros"],
+                                  None)
+    assert st == 1
+
+
+def test_quantize_clip_unsupported_group_size(lib):
+    # 512 is a valid RTN group size; the clipping search takes 32..256 only
+    assert lib.wq_quantize_clip_mse(FAKE, 4, 1024, 512, 0, FAKE, FAKE, FAKE, None) == 2

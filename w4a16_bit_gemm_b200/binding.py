@@ -50,6 +50,8 @@ def _load() -> ctypes.CDLL:
     lib.wq_status_string.restype = ctypes.c_char_p
     lib.wq_quantize_rtn.argtypes = [P, i64, i64, i32, i32, P, P, P, P]
     lib.wq_quantize_rtn.restype = ctypes.c_int
+    lib.wq_quantize_clip_mse.argtypes = [P, i64, i64, i32, i32, P, P, P, P]
+    lib.wq_quantize_clip_mse.restype = ctypes.c_int
     lib.wq_dequantize.argtypes = [P, P, P, i64, i64, i32, i32, P, P]
     lib.wq_dequantize.restype = ctypes.c_int
     lib.wq_linear_w4a16.argtypes = [P, i64, P, P, P, i64, i64, i32, i32, P, i32, P, sz, P]
@@ -100,6 +102,11 @@ def _require_cuda(*ts):
 def wq_quantize_rtn(W, d_out, d_in, group_size, symmetric, qweight, scales, zeros, stream=None) -> int:
     return lib.wq_quantize_rtn(_ptr(W), d_out, d_in, group_size, int(symmetric), _ptr(qweight), _ptr(scales),
                                _ptr(zeros), _stream(stream))
+
+
+def wq_quantize_clip_mse(W, d_out, d_in, group_size, symmetric, qweight, scales, zeros, stream=None) -> int:
+    return lib.wq_quantize_clip_mse(_ptr(W), d_out, d_in, group_size, int(symmetric), _ptr(qweight),
+                                    _ptr(scales), _ptr(zeros), _stream(stream))
 
 
 def wq_dequantize(qweight, scales, zeros, d_out, d_in, group_size, symmetric, W_hat, stream=None) -> int:
@@ -171,6 +178,23 @@ def quantize_rtn(W: torch.Tensor, group_size: int = 128, symmetric: bool = False
         out = alloc_packed(d_out, d_in, group_size, symmetric, W.device)
     _check(wq_quantize_rtn(W, d_out, d_in, group_size, symmetric, out.qweight, out.scales, out.zeros, stream),
            "wq_quantize_rtn")
+    return out
+
+
+def quantize_clip_mse(W: torch.Tensor, group_size: int = 128, symmetric: bool = False,
+                      out: PackedLinear | None = None, stream=None) -> PackedLinear:
+    """Group-wise quantization with the per-group MSE-optimal clipping search;
+    same artifact format as quantize_rtn."""
+    _require_cuda(W)
+    if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D bf16 CUDA tensor")
+    d_out, d_in = W.shape
+    if out is None:
+        if d_in % group_size != 0:
+            raise ValueError("group_size must divide d_in")
+        out = alloc_packed(d_out, d_in, group_size, symmetric, W.device)
+    _check(wq_quantize_clip_mse(W, d_out, d_in, group_size, symmetric, out.qweight, out.scales, out.zeros, stream),
+           "wq_quantize_clip_mse")
     return out
 
 

@@ -420,6 +420,108 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_kernel(
     }
 }
 
+// ------------------------------------------------------------------------
+// MSE-optimal clipping per group ("LLM Quantization: GPTQ, AWQ, SmoothQuant,
+// FP8, KV Cache (7/10)", Clipping Trade-off; "Quantization Algorithms" notes,
+// calibration 4, MSE-optimal argmin ||x - x_dq||^2 per group).
+// Candidate i shrinks the group's RTN range by alpha_i = fl32((20 - i) / 20),
+// i = 0..10; scale, zero and codes follow the RTN formulas on that range (the
+// exact scale_zero / encode path).  The candidate's error is
+// sum_k (x_k - x_hat_k)^2 over finite x_k, x_hat_k the bf16 dequant, in fp64
+// (difference, then the square rounded once, then the add; no fused
+// multiply-add), summed sequentially over each lane's 8 consecutive weights
+// and then by an xor butterfly over the group's L = g/8 lanes, i.e. a
+// pairwise tree over the 8-weight runs in index order -- the same operations
+// in the same order as the oracle, so the choice is identical.  The smallest error
+// wins; ties keep the smaller i.  alpha_0 = 1 reproduces RTN.
+// ------------------------------------------------------------------------
+constexpr int kClipCandidates = 11;
+
+// Exact codes (offset by nothing: q in [q_min, q_max]) of 8 values.
+__device__ __forceinline__ void codes8(const float v[8], const ScaleZero& sz, bool symmetric, int q[8]) {
+    const float s = __half2float(__ushort_as_half(sz.s16));
+    const float rcp = __frcp_rn(s);
+    const float qmin = symmetric ? -8.0f : 0.0f;
+    const float qmax = symmetric ? 7.0f : 15.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (isnan(v[i])) {
+            q[i] = sz.z;
+        } else {
+            const float t = rint_quotient(v[i], s, rcp);
+            q[i] = (int)fminf(fmaxf(__fadd_rn(t, (float)sz.z), qmin), qmax);
+        }
+    }
+}
+
+template <int L>
+__global__ void __launch_bounds__(kQuantThreads) quantize_clip_kernel(
+    const uint4* __restrict__ W, int64_t nseg, int symmetric, uint32_t* __restrict__ qweight,
+    uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros, uint32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const bool sym = symmetric != 0;
+    bool nonfinite = false, range = false;
+    const int64_t stride = (int64_t)gridDim.x * kQuantThreads;
+    for (int64_t base = (int64_t)blockIdx.x * kQuantThreads + threadIdx.x; base - threadIdx.x < nseg;
+         base += stride) {
+        const int64_t seg = base;
+        const uint4 raw = seg < nseg ? ld_nc_v4(W + seg) : make_uint4(0, 0, 0, 0);
+        float v[8];
+        unpack_bf16x8(raw, v);
+        float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            nonfinite |= !isfinite(v[i]);
+            lo = fminf(lo, v[i]);  // NaN is skipped (minNum / maxNum)
+            hi = fmaxf(hi, v[i]);
+        }
+#pragma unroll
+        for (int o = 1; o < L; o <<= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        double best_err = 0.0;
+        uint32_t best_word = 0;
+        ScaleZero best_sz = {0x3c00u, 0, false};
+        for (int i = 0; i < kClipCandidates; ++i) {
+            const float alpha = __fdiv_rn((float)(20 - i), 20.0f);
+            const ScaleZero sz = scale_zero(__fmul_rn(alpha, lo), __fmul_rn(alpha, hi), sym);
+            int q[8];
+            codes8(v, sz, sym, q);
+            const float s = __half2float(__ushort_as_half(sz.s16));
+            double err = 0.0;
+            uint32_t word = 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                word |= ((uint32_t)q[k] & 0xfu) << (4 * k);
+                const float xh = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s, (float)(q[k] - sz.z))));
+                const double e = __dsub_rn((double)v[k], (double)xh);
+                if (isfinite(v[k])) err = __dadd_rn(err, __dmul_rn(e, e));  // no fused multiply-add
+            }
+#pragma unroll
+            for (int o = 1; o < L; o <<= 1) err = __dadd_rn(err, __shfl_xor_sync(0xffffffffu, err, o));
+            if (i == 0 || err < best_err) {
+                best_err = err;
+                best_word = word;
+                best_sz = sz;
+            }
+        }
+        if (seg < nseg) {
+            range |= best_sz.range;
+            qweight[seg] = best_word;
+            if ((lane & (L - 1)) == 0) {
+                const int64_t gi = seg / L;
+                scales[gi] = best_sz.s16;
+                if (!sym) zeros[gi] = __half_as_ushort(__int2half_rn(best_sz.z));
+            }
+        }
+    }
+    const unsigned bad_nf = __ballot_sync(0xffffffffu, nonfinite);
+    const unsigned bad_rg = __ballot_sync(0xffffffffu, range);
+    if (lane == 0 && (bad_nf | bad_rg))
+        raise_flag(status, (bad_nf ? kFlagNonfinite : 0u) | (bad_rg ? kFlagRange : 0u));
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric,
@@ -458,6 +560,36 @@ cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, i
         const int64_t blocks = (ngroups + warps_per_block - 1) / warps_per_block;
         quantize_large_group_kernel<<<blocks, kQuantThreads, 0, stream>>>(W4, ngroups, g, symmetric, qweight, scales,
                                                                            zeros, status);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_clip(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric,
+                                 uint32_t* qweight, uint16_t* scales, uint16_t* zeros, uint32_t* status,
+                                 int num_sms, cudaStream_t stream) {
+    const int64_t nseg = d_out * d_in / 8;
+    int64_t blocks = (nseg + kQuantThreads - 1) / kQuantThreads;
+    if (blocks > (int64_t)num_sms * 16) blocks = (int64_t)num_sms * 16;
+    const uint4* W4 = static_cast<const uint4*>(W);
+    switch (g) {
+        case 32:
+            quantize_clip_kernel<4><<<blocks, kQuantThreads, 0, stream>>>(W4, nseg, symmetric, qweight, scales,
+                                                                           zeros, status);
+            break;
+        case 64:
+            quantize_clip_kernel<8><<<blocks, kQuantThreads, 0, stream>>>(W4, nseg, symmetric, qweight, scales,
+                                                                           zeros, status);
+            break;
+        case 128:
+            quantize_clip_kernel<16><<<blocks, kQuantThreads, 0, stream>>>(W4, nseg, symmetric, qweight, scales,
+                                                                            zeros, status);
+            break;
+        case 256:
+            quantize_clip_kernel<32><<<blocks, kQuantThreads, 0, stream>>>(W4, nseg, symmetric, qweight, scales,
+                                                                            zeros, status);
+            break;
+        default:
+            return cudaErrorNotSupported;
     }
     return cudaGetLastError();
 }

@@ -155,6 +155,21 @@ wq_status wq_quantize_rtn(const void* W_bf16, int64_t d_out, int64_t d_in, int32
     return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
+wq_status wq_quantize_clip_mse(const void* W_bf16, int64_t d_out, int64_t d_in, int32_t group_size,
+                               int32_t symmetric, uint32_t* qweight, void* scales_fp16, void* zeros_fp16,
+                               void* stream) {
+    if (!W_bf16 || !aligned(W_bf16, 16)) return WQ_ERR_INVALID_ARG;
+    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
+    if (v != WQ_OK) return v;
+    if (group_size != 32 && group_size != 64 && group_size != 128 && group_size != 256) return WQ_ERR_UNSUPPORTED;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    cudaError_t e = launch_quantize_clip(W_bf16, d_out, d_in, group_size, symmetric, qweight,
+                                         static_cast<uint16_t*>(scales_fp16), static_cast<uint16_t*>(zeros_fp16),
+                                         st.status, st.num_sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
 wq_status wq_dequantize(const uint32_t* qweight, const void* scales_fp16, const void* zeros_fp16, int64_t d_out,
                         int64_t d_in, int32_t group_size, int32_t symmetric, void* W_hat_bf16, void* stream) {
     wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);

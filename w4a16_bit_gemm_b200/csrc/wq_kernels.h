@@ -10,6 +10,12 @@ namespace wq {
 cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric, uint32_t* qweight,
                             uint16_t* scales, uint16_t* zeros, uint32_t* status, int num_sms, cudaStream_t stream);
 
+// Quantize with the per-group MSE-optimal clipping search; g in {32, 64, 128, 256}
+// (cudaErrorNotSupported otherwise).
+cudaError_t launch_quantize_clip(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric,
+                                 uint32_t* qweight, uint16_t* scales, uint16_t* zeros, uint32_t* status,
+                                 int num_sms, cudaStream_t stream);
+
 cudaError_t launch_dequantize(const uint32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
                               int64_t d_out, int64_t d_in, int g, int symmetric, void* W_hat, int num_sms,
                               cudaStream_t stream);
