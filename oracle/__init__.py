@@ -118,6 +118,10 @@ def _load(path: str | None = None):
             lib.wqo_quantize_group_range.restype = ctypes.c_uint32
             lib.wqo_group_sq_error.argtypes = [P, i64, P, ctypes.c_uint16, ctypes.c_int32]
             lib.wqo_group_sq_error.restype = ctypes.c_double
+            lib.wqo_awq_search.argtypes = [P, i64, i64, P, i64, i64, i32, P, P, P, P, P, P, i32]
+            lib.wqo_awq_search.restype = i32
+            lib.wqo_awq_scales.argtypes = [P, i64, i64, ctypes.c_double, P]
+            lib.wqo_awq_scales.restype = None
             lib.wqo_clip_alpha.argtypes = [i32]
             lib.wqo_clip_alpha.restype = ctypes.c_float
             for nm in ("wqo_f32_to_f16_array", "wqo_f32_to_bf16_array", "wqo_f16_to_f32_array"):
@@ -266,6 +270,46 @@ def group_sq_error(x_bits: np.ndarray, codes: np.ndarray, s16: int, z: int) -> f
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     codes = np.ascontiguousarray(codes, dtype=np.int32)
     return float(_load().wqo_group_sq_error(_ptr(x_bits), x_bits.shape[0], _ptr(codes), s16, z))
+
+
+AWQ_ALPHAS = 11
+
+
+def awq_search(W_bits: np.ndarray, X_bits: np.ndarray, group_size: int = 128, symmetric: bool = False,
+               nthreads: int | None = None):
+    """AWQ per-input-channel scaling search ([P2] AWQ procedure).
+
+    W_bits bf16 [N, K], X_bits bf16 calibration [T, K].  Returns ``(codes,
+    scales, zeros or None, s_bf16 [K], losses [11], best)``: the RTN artifact
+    of W diag(s) for the best alpha = best / 10, its per-channel scales s
+    (bf16 bits; the linear layer then takes x / s) and every alpha's loss.
+    """
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    N, K = W_bits.shape
+    T = X_bits.shape[0]
+    G = K // group_size
+    codes = np.empty((N, K), np.int32)
+    scales = np.empty((N, G), np.uint16)
+    zeros = None if symmetric else np.empty((N, G), np.uint16)
+    s = np.empty(K, np.uint16)
+    losses = np.empty(AWQ_ALPHAS, np.float64)
+    best = ctypes.c_int32(-1)
+    rc = _load().wqo_awq_search(_ptr(W_bits), N, K, _ptr(X_bits), T, group_size, int(symmetric), _ptr(codes),
+                                _ptr(scales), _ptr(zeros) if zeros is not None else None, _ptr(s), _ptr(losses),
+                                ctypes.cast(ctypes.pointer(best), ctypes.c_void_p), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle AWQ search rejected its arguments")
+    return codes, scales, zeros, s, losses, int(best.value)
+
+
+def awq_scales(X_bits: np.ndarray, alpha: float) -> np.ndarray:
+    """Per-channel AWQ scales (bf16 bits [K]) for one alpha."""
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    T, K = X_bits.shape
+    s = np.empty(K, np.uint16)
+    _load().wqo_awq_scales(_ptr(X_bits), T, K, float(alpha), _ptr(s))
+    return s
 
 
 def pack4(codes: np.ndarray) -> np.ndarray:

@@ -495,6 +495,134 @@ int wqo_quantize_clip(const uint16_t* W, int64_t d_out, int64_t d_in, int64_t g,
 }
 
 /* ------------------------------------------------------------------------ */
+/* AWQ: activation-aware per-input-channel scaling                           */
+/* [P2 "AWQ" procedure]: per-channel mean |x| over a calibration batch; for   */
+/* alpha in {0, 0.1, ..., 1.0}: s = mean|x|^alpha / geomean, W' = W diag(s),  */
+/* loss = ||W X - Q(W') (X / s)||; keep the argmin; s^-1 is fused into the    */
+/* previous layer [P1 "AWQ": protect salient channels found from activation   */
+/* statistics through per-channel scaling].                                  */
+/* Readings (the pages leave them open):                                     */
+/*  - m_j = (sum_t |X[t,j]|) / T in fp64 (exact sum of bf16 values), floored  */
+/*    at 2^-30;                                                              */
+/*  - alpha_i = i / 10 (fp64), i = 0..10;                                     */
+/*  - s_j = bf16_rn(fl32(exp(alpha (ln m_j - mean_j ln m_j)))), i.e. m^alpha  */
+/*    over its geometric mean (fp64), rounded to fp32 then bf16, so that the  */
+/*    two products below are one multiply or divide and one rounding each;    */
+/*  - W'[n,j] = bf16_rn(fl32(W[n,j] s_j)); X'[t,j] = bf16_rn(fl32(X[t,j]/s_j)); */
+/*  - Q(W') is the RTN artifact of W' (quantize_group) and its dequant;        */
+/*  - loss = sum_{t,n} (Y[t,n] - Y'[t,n])^2 with Y = X W^T and Y' = X' Q(W')^T  */
+/*    in fp64; the smallest loss wins, ties to the smaller alpha.             */
+/* alpha = 0 gives s = 1, i.e. plain RTN of W.                                */
+/* ------------------------------------------------------------------------ */
+
+#define WQO_AWQ_ALPHAS 11
+
+int wqo_dequantize(const int32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,
+                   int64_t d_in, int64_t g, uint16_t* W_hat, int nthreads);
+
+/* Y[t][n] = sum_j A[t][j] B[n][j] in fp64 for bf16 inputs (rows of A: T, rows of B: N). */
+typedef struct {
+    const uint16_t *A, *B;
+    int64_t T, N, K;
+    double* Y;
+} gemm_ctx;
+
+static void gemm_rows(void* vctx, int64_t t0, int64_t t1, uint32_t* flags) {
+    gemm_ctx* c = (gemm_ctx*)vctx;
+    (void)flags;
+    for (int64_t t = t0; t < t1; ++t)
+        for (int64_t n = 0; n < c->N; ++n) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < c->K; ++j)
+                acc += (double)wqo_bf16_to_f32(c->A[t * c->K + j]) * (double)wqo_bf16_to_f32(c->B[n * c->K + j]);
+            c->Y[t * c->N + n] = acc;
+        }
+}
+
+static void gemm_bf16_f64(const uint16_t* A, int64_t T, const uint16_t* B, int64_t N, int64_t K, double* Y,
+                          int nthreads) {
+    gemm_ctx c = {A, B, T, N, K, Y};
+    run_rows(gemm_rows, &c, T, nthreads);
+}
+
+/* Per-channel scales for one alpha (bf16 bits). */
+void wqo_awq_scales(const uint16_t* X, int64_t T, int64_t K, double alpha, uint16_t* s_out) {
+    double* lnm = (double*)malloc(sizeof(double) * (size_t)K);
+    double mean_ln = 0.0;
+    for (int64_t j = 0; j < K; ++j) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < T; ++t) acc += fabs((double)wqo_bf16_to_f32(X[t * K + j]));
+        double m = acc / (double)T;
+        if (m < 0x1p-30) m = 0x1p-30;
+        lnm[j] = log(m);
+    }
+    for (int64_t j = 0; j < K; ++j) mean_ln += lnm[j];
+    mean_ln /= (double)K;
+    for (int64_t j = 0; j < K; ++j) {
+#if WQO_MUTANT == 11 /* mistake: scales inverted (divide instead of multiply) */
+        s_out[j] = wqo_f32_to_bf16((float)exp(-alpha * (lnm[j] - mean_ln)));
+#else
+        s_out[j] = wqo_f32_to_bf16((float)exp(alpha * (lnm[j] - mean_ln)));
+#endif
+    }
+    free(lnm);
+}
+
+/* Search; outputs the artifact of the best alpha, its scales s (bf16 [K]),
+ * the 11 losses and the best index.  Returns 0, or -1 on bad arguments. */
+int wqo_awq_search(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t T, int64_t g,
+                   int symmetric, int32_t* codes, uint16_t* scales, uint16_t* zeros, uint16_t* s_best,
+                   double* losses, int32_t* best, int nthreads) {
+    if (!W || !X || !codes || !scales || !s_best || N < 1 || K < 1 || T < 1 || g < 1 || K % g != 0) return -1;
+    if (!symmetric && !zeros) return -1;
+    const int64_t G = K / g;
+    uint16_t* s = (uint16_t*)malloc(2 * (size_t)K);
+    uint16_t* Wp = (uint16_t*)malloc(2 * (size_t)(N * K));
+    uint16_t* Xp = (uint16_t*)malloc(2 * (size_t)(T * K));
+    uint16_t* Wh = (uint16_t*)malloc(2 * (size_t)(N * K));
+    int32_t* cc = (int32_t*)malloc(4 * (size_t)(N * K));
+    uint16_t* sc = (uint16_t*)malloc(2 * (size_t)(N * G));
+    uint16_t* zc = (uint16_t*)malloc(2 * (size_t)(N * G));
+    double* Y = (double*)malloc(sizeof(double) * (size_t)(T * N));
+    double* Yp = (double*)malloc(sizeof(double) * (size_t)(T * N));
+    gemm_bf16_f64(X, T, W, N, K, Y, nthreads);
+    double best_loss = 0.0;
+    int best_i = -1;
+    for (int i = 0; i < WQO_AWQ_ALPHAS; ++i) {
+        double alpha = (double)i / 10.0;
+        wqo_awq_scales(X, T, K, alpha, s);
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t j = 0; j < K; ++j)
+                Wp[n * K + j] = wqo_f32_to_bf16(wqo_bf16_to_f32(W[n * K + j]) * wqo_bf16_to_f32(s[j]));
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t j = 0; j < K; ++j)
+                Xp[t * K + j] = wqo_f32_to_bf16(wqo_bf16_to_f32(X[t * K + j]) / wqo_bf16_to_f32(s[j]));
+        uint32_t fl;
+        wqo_quantize(Wp, N, K, g, 4, symmetric, 0, cc, sc, symmetric ? NULL : zc, &fl, nthreads);
+        wqo_dequantize(cc, sc, symmetric ? NULL : zc, N, K, g, Wh, nthreads);
+        gemm_bf16_f64(Xp, T, Wh, N, K, Yp, nthreads);
+        double loss = 0.0;
+        for (int64_t q = 0; q < T * N; ++q) {
+            double d = Y[q] - Yp[q];
+            loss += d * d;
+        }
+        if (losses) losses[i] = loss;
+        if (best_i < 0 || loss < best_loss) {
+            best_i = i;
+            best_loss = loss;
+            for (int64_t q = 0; q < N * K; ++q) codes[q] = cc[q];
+            for (int64_t q = 0; q < N * G; ++q) scales[q] = sc[q];
+            if (!symmetric)
+                for (int64_t q = 0; q < N * G; ++q) zeros[q] = zc[q];
+            for (int64_t j = 0; j < K; ++j) s_best[j] = s[j];
+        }
+    }
+    if (best) *best = best_i;
+    free(s); free(Wp); free(Xp); free(Wh); free(cc); free(sc); free(zc); free(Y); free(Yp);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Packing (4-bit only): 8 nibbles per uint32, low nibble first.             */
 /* ------------------------------------------------------------------------ */
 

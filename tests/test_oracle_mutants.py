@@ -2,10 +2,11 @@
 in with -DWQO_MUTANT=k) must fail at least one pin, and the real oracle must
 pass the same pins.  This shows the pins constrain every step: statistics,
 scale, zero point, rounding, packing, dequantization, the linear layer and
-the clipping search (error formula and selection)."""
+the clipping search (error formula and selection) and the AWQ scales."""
 import pytest
 
 import oracle
+from tests import test_oracle_awq_pins as awq_pins
 from tests import test_oracle_clip_pins as clip_pins
 from tests import test_oracle_pins as pins
 
@@ -22,6 +23,8 @@ PINS = [
     clip_pins.test_error_formula_is_the_exact_sum_of_squares,
     clip_pins.test_choice_is_the_exact_argmin,
     clip_pins.test_never_worse_than_rtn,
+    awq_pins.test_scales_follow_the_page_formula,
+    awq_pins.test_losses_and_choice_recomputed_independently,
 ]
 
 MUTANTS = {
@@ -34,6 +37,7 @@ MUTANTS = {
     7: "high nibble first",
     9: "clip search sums absolute errors",
     10: "clip search keeps the largest error",
+    11: "AWQ scales inverted",
 }
 
 
