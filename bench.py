@@ -327,6 +327,31 @@ def run_ours(args, dist: Dist):
                                       "frac_of_measured_hbm": qb / tqc / 1e9 / hbm,
                                       "sq_error_vs_rtn": err_clip / err_rtn}
     del gqc, p_clip, Wd
+    # AWQ per-input-channel scaling search (11 alphas) with 512 calibration
+    # tokens carrying the 0.1% x50 activation channels; eager launches (the
+    # search holds ~70 launches, ~1 ms of device work, so the host keeps ahead)
+    T_CAL = 512
+    Xc = syn.activations(T_CAL, D, 21, 2, "cuda", channel_outlier_frac=0.001)
+    ws = torch.empty(b.wq_awq_workspace_bytes(D, D, T_CAL, G128), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        r_awq = b.awq_search(W, Xc, workspace=ws)
+    torch.cuda.synchronize()
+    dist.barrier()
+    asteps = 5
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(asteps):
+        r_awq = b.awq_search(W, Xc, workspace=ws)
+    ev1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    ta = dist.max(ev0.elapsed_time(ev1) / 1e3) / asteps
+    a_best = int(r_awq.best.item())
+    a_losses = r_awq.losses.cpu()
+    secondary["awq_search"] = {"shape": "4096x4096", "calib_tokens": T_CAL, "alphas": 11,
+                               "ms_per_search": ta * 1e3, "alpha": a_best / 10.0,
+                               "loss_vs_rtn": float(a_losses[a_best] / a_losses[0])}
+    del r_awq, ws, Xc
     What = [torch.empty(D, D, dtype=torch.bfloat16, device="cuda") for _ in range(QC)]
 
     def dfn():

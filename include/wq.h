@@ -191,6 +191,62 @@ wq_status wq_linear_w4a16(const void* X_bf16, int64_t M, const uint32_t* qweight
 size_t wq_linear_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in);
 
 /*
+ * wq_awq_search -- activation-aware per-input-channel scaling (AWQ), then
+ * group-wise RTN of the scaled weights ("Quantization Algorithms" study
+ * notes, AWQ section and its procedure; "LLM Quantization: GPTQ, AWQ,
+ * SmoothQuant, FP8, KV Cache (7/10)", AWQ section).  The scaling identity
+ * W x = (W diag(s)) (x / s) moves quantization error away from the input
+ * channels whose activations are large.
+ *
+ * For a calibration batch X[T][d_in]:
+ *   m_j  = (sum_t |X[t][j]|) / T in fp64 (sequential in t), floored at 2^-30;
+ *   for alpha_i = i / 10, i = 0..10:
+ *     s_j  = bf16_rn(fl32(exp(alpha_i (ln m_j - mean_j ln m_j))))
+ *            (mean|x|^alpha divided by its geometric mean over the channels);
+ *     W'   = bf16_rn(fl32(W[n][j] s_j)),  X' = bf16_rn(fl32(X[t][j] / s_j));
+ *     Q(W') = the wq_quantize_rtn artifact of W';
+ *     loss_i = sum_{t,n} (Y[t][n] - Y'[t][n])^2 in fp64, with Y = X W^T
+ *            (fp32 accumulation, a library GEMM) and Y' = X' Q(W')^T from
+ *            wq_linear_w4a16 with fp32 output;
+ *   the smallest loss is kept (ties: the smaller i).  alpha_0 = 0 gives s = 1,
+ *   i.e. plain RTN.  The losses are deterministic run to run.
+ *
+ *   W_bf16      [d_out][d_in] bf16 weights, input.  16-byte aligned.
+ *   X_bf16      [T][d_in] bf16 calibration activations, input.  16-byte aligned.
+ *   T           calibration tokens, 1 .. 2^31 - 1.
+ *   group_size, symmetric, qweight, scales_fp16, zeros_fp16:
+ *               as wq_quantize_rtn; the output artifact is that of W' for
+ *               the kept alpha.
+ *   s_bf16      [d_in] bf16 output: the kept per-channel scales.  The layer
+ *               then computes Y = (X / s) Q(W')^T: wq_awq_scale_activations
+ *               divides X, or the division is folded into the producer of X.
+ *   losses      device fp64 [11] output, or NULL.
+ *   best        device int32 output (the kept i), or NULL.
+ *   workspace   device scratch of at least wq_awq_workspace_bytes(...)
+ *               bytes, 256-byte aligned, owned by the caller.
+ * All work is queued on `stream`; the call does not synchronize.
+ * Errors: WQ_ERR_INVALID_ARG as wq_quantize_rtn plus a missing or small
+ * workspace or a bad T; WQ_ERR_CUDA if a launch or the library GEMM fails.
+ * Device flags: as wq_quantize_rtn, from every candidate's quantization.
+ */
+wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const void* X_bf16, int64_t T,
+                        int32_t group_size, int32_t symmetric, uint32_t* qweight, void* scales_fp16,
+                        void* zeros_fp16, void* s_bf16, double* losses, int32_t* best, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* Scratch bytes wq_awq_search needs (0 for invalid shapes). */
+size_t wq_awq_workspace_bytes(int64_t d_out, int64_t d_in, int64_t T, int32_t group_size);
+
+/*
+ * wq_awq_scale_activations -- X'[t][j] = bf16_rn(fl32(X[t][j] / s_j)), the
+ * activation side of the AWQ scaling identity.  X_bf16 and Xp_bf16 are
+ * [T][d_in] bf16, 16-byte aligned (they may not overlap unless equal);
+ * s_bf16 is [d_in] bf16.  d_in must be a multiple of 8.
+ */
+wq_status wq_awq_scale_activations(const void* X_bf16, int64_t T, int64_t d_in, const void* s_bf16,
+                                   void* Xp_bf16, void* stream);
+
+/*
  * wq_get_device_error -- synchronize `stream`, read and clear the device
  * status word of the current device.  *flags receives the WQ_DEVFLAG_* bits
  * (may be NULL).  Returns WQ_OK when no bit was set, otherwise the status of

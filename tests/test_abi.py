@@ -27,7 +27,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for n in ("wq_quantize_rtn", "wq_quantize_clip_mse", "wq_dequantize", "wq_linear_w4a16", "wq_linear_workspace_bytes",
+    for n in ("wq_quantize_rtn", "wq_quantize_clip_mse", "wq_awq_search", "wq_awq_workspace_bytes",
+              "wq_awq_scale_activations", "wq_dequantize", "wq_linear_w4a16", "wq_linear_workspace_bytes",
               "wq_get_device_error", "wq_status_string", "wq_abi_version"):
         assert n in names
 
@@ -101,3 +102,31 @@ def test_quantize_clip_rejects(lib, case):
 def test_quantize_clip_unsupported_group_size(lib):
     # 512 is a valid RTN group size; the clipping search takes 32..256 only
     assert lib.wq_quantize_clip_mse(FAKE, 4, 1024, 512, 0, FAKE, FAKE, FAKE, None) == 2
+
+
+@pytest.mark.parametrize("case", [
+    dict(W=None), dict(X=None), dict(X=FAKE + 8), dict(s=None), dict(T=0), dict(ws=None), dict(wsb=16),
+    dict(ws=FAKE + 16), dict(d_in=1000), dict(zeros=None), dict(sym=1), dict(losses=FAKE + 4),
+])
+def test_awq_search_rejects(lib, case):
+    a = dict(W=FAKE, d_out=4, d_in=256, X=FAKE, T=8, g=128, sym=0, q=FAKE, sc=FAKE, zeros=FAKE, s=FAKE,
+             losses=None, best=None, ws=FAKE, wsb=1 << 30)
+    a.update(case)
+    st = lib.wq_awq_search(a["W"], a["d_out"], a["d_in"], a["X"], a["T"], a["g"], a["sym"], a["q"], a["sc"],
+                           a["zeros"], a["s"], a["losses"], a["best"], a["ws"], a["wsb"], None)
+    assert st == 1
+
+
+def test_awq_workspace_query(lib):
+    n = lib.wq_awq_workspace_bytes(4096, 4096, 512, 128)
+    # W' and X' (bf16), the candidate artifact, two fp32 outputs, at least
+    assert n >= 4096 * 4096 * 2 + 4096 * 2048 + 512 * 4096 * 2 + 2 * 512 * 4096 * 4
+    assert lib.wq_awq_workspace_bytes(4, 1000, 8, 128) == 0
+    assert lib.wq_awq_workspace_bytes(0, 256, 8, 128) == 0
+
+
+def test_awq_scale_activations_rejects(lib):
+    assert lib.wq_awq_scale_activations(None, 4, 256, FAKE, FAKE, None) == 1
+    assert lib.wq_awq_scale_activations(FAKE, 0, 256, FAKE, FAKE, None) == 1
+    assert lib.wq_awq_scale_activations(FAKE, 4, 252, FAKE, FAKE, None) == 1
+    assert lib.wq_awq_scale_activations(FAKE + 8, 4, 256, FAKE, FAKE, None) == 1

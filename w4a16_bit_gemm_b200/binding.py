@@ -58,6 +58,12 @@ def _load() -> ctypes.CDLL:
     lib.wq_linear_w4a16.restype = ctypes.c_int
     lib.wq_linear_workspace_bytes.argtypes = [i64, i64, i64]
     lib.wq_linear_workspace_bytes.restype = sz
+    lib.wq_awq_search.argtypes = [P, i64, i64, P, i64, i32, i32, P, P, P, P, P, P, P, sz, P]
+    lib.wq_awq_search.restype = ctypes.c_int
+    lib.wq_awq_workspace_bytes.argtypes = [i64, i64, i64, i32]
+    lib.wq_awq_workspace_bytes.restype = sz
+    lib.wq_awq_scale_activations.argtypes = [P, i64, i64, P, P, P]
+    lib.wq_awq_scale_activations.restype = ctypes.c_int
     lib.wq_get_device_error.argtypes = [P, P]
     lib.wq_get_device_error.restype = ctypes.c_int
     lib.wq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
@@ -118,6 +124,21 @@ def wq_linear_w4a16(X, M, qweight, scales, zeros, d_out, d_in, group_size, symme
                     workspace_bytes=0, stream=None) -> int:
     return lib.wq_linear_w4a16(_ptr(X), M, _ptr(qweight), _ptr(scales), _ptr(zeros), d_out, d_in, group_size,
                                int(symmetric), _ptr(Y), y_dtype, _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def wq_awq_search(W, d_out, d_in, X, T, group_size, symmetric, qweight, scales, zeros, s, losses, best, workspace,
+                  workspace_bytes, stream=None) -> int:
+    return lib.wq_awq_search(_ptr(W), d_out, d_in, _ptr(X), T, group_size, int(symmetric), _ptr(qweight),
+                             _ptr(scales), _ptr(zeros), _ptr(s), _ptr(losses), _ptr(best), _ptr(workspace),
+                             workspace_bytes, _stream(stream))
+
+
+def wq_awq_workspace_bytes(d_out, d_in, T, group_size) -> int:
+    return int(lib.wq_awq_workspace_bytes(d_out, d_in, T, group_size))
+
+
+def wq_awq_scale_activations(X, T, d_in, s, Xp, stream=None) -> int:
+    return lib.wq_awq_scale_activations(_ptr(X), T, d_in, _ptr(s), _ptr(Xp), _stream(stream))
 
 
 def wq_linear_workspace_bytes(M, d_out, d_in) -> int:
@@ -195,6 +216,55 @@ def quantize_clip_mse(W: torch.Tensor, group_size: int = 128, symmetric: bool = 
         out = alloc_packed(d_out, d_in, group_size, symmetric, W.device)
     _check(wq_quantize_clip_mse(W, d_out, d_in, group_size, symmetric, out.qweight, out.scales, out.zeros, stream),
            "wq_quantize_clip_mse")
+    return out
+
+
+class AWQResult:
+    """Output of awq_search: the artifact of W diag(s), the per-input-channel
+    scales s (bf16 [d_in]), the 11 losses (fp64, device) and the kept index
+    (int32, device; alpha = index / 10)."""
+
+    def __init__(self, packed, s, losses, best):
+        self.packed = packed
+        self.s = s
+        self.losses = losses
+        self.best = best
+
+
+def awq_search(W: torch.Tensor, X: torch.Tensor, group_size: int = 128, symmetric: bool = False,
+               workspace: torch.Tensor | None = None, stream=None) -> AWQResult:
+    """AWQ per-input-channel scaling search over alpha = 0, 0.1, ..., 1 on the
+    calibration activations X[T, d_in], then RTN of W diag(s)."""
+    _require_cuda(W, X)
+    if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D bf16 CUDA tensor")
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or not X.is_contiguous() or X.shape[1] != W.shape[1]:
+        raise ValueError("X must be a contiguous [T, d_in] bf16 CUDA tensor")
+    d_out, d_in = W.shape
+    T = X.shape[0]
+    if d_in % group_size != 0:
+        raise ValueError("group_size must divide d_in")
+    out = alloc_packed(d_out, d_in, group_size, symmetric, W.device)
+    s = torch.empty(d_in, dtype=torch.bfloat16, device=W.device)
+    losses = torch.empty(11, dtype=torch.float64, device=W.device)
+    best = torch.empty(1, dtype=torch.int32, device=W.device)
+    need = wq_awq_workspace_bytes(d_out, d_in, T, group_size)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    _check(wq_awq_search(W, d_out, d_in, X, T, group_size, symmetric, out.qweight, out.scales, out.zeros, s, losses,
+                         best, workspace, workspace.numel() * workspace.element_size(), stream), "wq_awq_search")
+    return AWQResult(out, s, losses, best)
+
+
+def awq_scale_activations(X: torch.Tensor, s: torch.Tensor, out: torch.Tensor | None = None,
+                          stream=None) -> torch.Tensor:
+    """X' = bf16(X / s) per input channel (the activation side of AWQ)."""
+    _require_cuda(X, s)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or not X.is_contiguous() or s.numel() != X.shape[1]:
+        raise ValueError("X must be a contiguous [T, d_in] bf16 CUDA tensor and s a [d_in] bf16 tensor")
+    if out is None:
+        out = torch.empty_like(X)
+    _check(wq_awq_scale_activations(X, X.shape[0], X.shape[1], s, out, stream), "wq_awq_scale_activations")
     return out
 
 

@@ -3,7 +3,8 @@
     python -m w4a16_bit_gemm_b200.build [--verbose-ptxas] [--force]
 
 Each .cu file under csrc/ is compiled to an object file in _build/ and linked
-into w4a16_bit_gemm_b200/libwq.so (CUDA runtime linked statically).
+into w4a16_bit_gemm_b200/libwq.so (CUDA runtime linked statically; cuBLAS
+dynamically, for the full-precision reference GEMM of the AWQ search).
 """
 from __future__ import annotations
 
@@ -22,6 +23,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libwq.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+CUDA_LIB = "/usr/local/cuda/lib64"
 
 
 def nvcc() -> str:
@@ -76,7 +78,8 @@ def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = False)
         raise RuntimeError("nvcc failed")
     if force or jobs or _stale(LIB, objs):
         tmp = LIB + ".tmp%d" % os.getpid()
-        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs]
+        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-lcublas",
+               "-Xlinker", "-rpath," + CUDA_LIB]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)

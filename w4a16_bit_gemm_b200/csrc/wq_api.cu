@@ -10,6 +10,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <cublas_v2.h>
 #include <mutex>
 
 #include "../../include/wq.h"
@@ -190,22 +191,14 @@ size_t wq_linear_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in) {
     return 0;
 }
 
-wq_status wq_linear_w4a16(const void* X_bf16, int64_t M, const uint32_t* qweight, const void* scales_fp16,
-                          const void* zeros_fp16, int64_t d_out, int64_t d_in, int32_t group_size, int32_t symmetric,
-                          void* Y, int32_t y_dtype, void* workspace, size_t workspace_bytes, void* stream) {
-    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
-    if (v != WQ_OK) return v;
-    if (!X_bf16 || !Y || !aligned(X_bf16, 16) || !aligned(Y, 16)) return WQ_ERR_INVALID_ARG;
-    if (M < 1 || M > (1ll << 31) - 1) return WQ_ERR_INVALID_ARG;
-    if (y_dtype != WQ_OUT_BF16 && y_dtype != WQ_OUT_FP32) return WQ_ERR_INVALID_ARG;
-    if (workspace_bytes < wq_linear_workspace_bytes(M, d_out, d_in)) return WQ_ERR_INVALID_ARG;
-    (void)workspace;
-    DeviceState st;
-    if ((v = device_state(&st)) != WQ_OK) return v;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+namespace {
+
+// The linear layer after argument checks: GEMV for M <= 16, tcgen05 GEMM above.
+cudaError_t run_linear(const DeviceState& st, const void* X_bf16, int64_t M, const uint32_t* qweight,
+                       const void* scales_fp16, const void* zeros_fp16, int64_t d_out, int64_t d_in,
+                       int32_t group_size, int32_t symmetric, void* Y, int32_t y_dtype, cudaStream_t s) {
     LaunchOptions opt;
     opt.pdl = pdl_enabled();
-    cudaError_t e;
     if (M <= 16) {
         GemvArgs a = {};
         a.X = X_bf16;
@@ -223,24 +216,163 @@ wq_status wq_linear_w4a16(const void* X_bf16, int64_t M, const uint32_t* qweight
             if ((1 << sh) == group_size) a.g_shift = sh;
         a.symmetric = symmetric;
         a.y_fp32 = y_dtype == WQ_OUT_FP32;
-        e = launch_gemv(qweight, a, st.num_sms, opt, s);
-    } else {
-        GemmArgs a = {};
-        a.X = X_bf16;
-        a.qweight = qweight;
-        a.scales = static_cast<const uint16_t*>(scales_fp16);
-        a.zeros = static_cast<const uint16_t*>(zeros_fp16);
-        a.Y = Y;
-        a.status = st.status;
-        a.M = (int)M;
-        a.N = (int)d_out;
-        a.K = (int)d_in;
-        a.g = group_size;
-        a.G = (int)(d_in / group_size);
-        a.symmetric = symmetric;
-        a.y_fp32 = y_dtype == WQ_OUT_FP32;
-        e = launch_gemm(a, st.num_sms, opt, s);
+        return launch_gemv(qweight, a, st.num_sms, opt, s);
     }
+    GemmArgs a = {};
+    a.X = X_bf16;
+    a.qweight = qweight;
+    a.scales = static_cast<const uint16_t*>(scales_fp16);
+    a.zeros = static_cast<const uint16_t*>(zeros_fp16);
+    a.Y = Y;
+    a.status = st.status;
+    a.M = (int)M;
+    a.N = (int)d_out;
+    a.K = (int)d_in;
+    a.g = group_size;
+    a.G = (int)(d_in / group_size);
+    a.symmetric = symmetric;
+    a.y_fp32 = y_dtype == WQ_OUT_FP32;
+    return launch_gemm(a, st.num_sms, opt, s);
+}
+
+}  // namespace
+
+wq_status wq_linear_w4a16(const void* X_bf16, int64_t M, const uint32_t* qweight, const void* scales_fp16,
+                          const void* zeros_fp16, int64_t d_out, int64_t d_in, int32_t group_size, int32_t symmetric,
+                          void* Y, int32_t y_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
+    if (v != WQ_OK) return v;
+    if (!X_bf16 || !Y || !aligned(X_bf16, 16) || !aligned(Y, 16)) return WQ_ERR_INVALID_ARG;
+    if (M < 1 || M > (1ll << 31) - 1) return WQ_ERR_INVALID_ARG;
+    if (y_dtype != WQ_OUT_BF16 && y_dtype != WQ_OUT_FP32) return WQ_ERR_INVALID_ARG;
+    if (workspace_bytes < wq_linear_workspace_bytes(M, d_out, d_in)) return WQ_ERR_INVALID_ARG;
+    (void)workspace;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    const cudaError_t e = run_linear(st, X_bf16, M, qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size,
+                                     symmetric, Y, y_dtype, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// AWQ search
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kAwqAlphas = 11;
+
+struct AwqWorkspace {
+    size_t wp, qa, sa, za, xp, yref, ya, lnm, red, scal, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+AwqWorkspace awq_workspace(int64_t N, int64_t K, int64_t T, int64_t g) {
+    AwqWorkspace w;
+    size_t o = 0;
+    const int64_t G = K / g;
+    w.wp = o;   o += align256((size_t)(N * K) * 2);
+    w.qa = o;   o += align256((size_t)(N * K) / 2);
+    w.sa = o;   o += align256((size_t)(N * G) * 2);
+    w.za = o;   o += align256((size_t)(N * G) * 2);
+    w.xp = o;   o += align256((size_t)(T * K) * 2);
+    w.yref = o; o += align256((size_t)(T * N) * 4);
+    w.ya = o;   o += align256((size_t)(T * N) * 4);
+    w.lnm = o;  o += align256((size_t)K * 8);
+    w.red = o;  o += align256((size_t)(awq_loss_partials() + 64) * 8);
+    w.scal = o; o += align256((size_t)K * 2);
+    w.total = o;
+    return w;
+}
+
+std::mutex g_blas_mu;
+cublasHandle_t g_blas[kMaxDevices] = {};
+
+}  // namespace
+
+size_t wq_awq_workspace_bytes(int64_t d_out, int64_t d_in, int64_t T, int32_t group_size) {
+    if (d_out < 1 || d_in < 1 || T < 1 || group_size < 1 || d_in % group_size != 0) return 0;
+    return awq_workspace(d_out, d_in, T, group_size).total;
+}
+
+wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const void* X_bf16, int64_t T,
+                        int32_t group_size, int32_t symmetric, uint32_t* qweight, void* scales_fp16,
+                        void* zeros_fp16, void* s_bf16, double* losses, int32_t* best, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
+    if (v != WQ_OK) return v;
+    if (!W_bf16 || !X_bf16 || !s_bf16 || !workspace || !aligned(W_bf16, 16) || !aligned(X_bf16, 16) ||
+        !aligned(s_bf16, 2) || !aligned(workspace, 256))
+        return WQ_ERR_INVALID_ARG;
+    if (T < 1 || T > (1ll << 31) - 1 || (d_in % 8) != 0) return WQ_ERR_INVALID_ARG;
+    if ((losses && !aligned(losses, 8)) || (best && !aligned(best, 4))) return WQ_ERR_INVALID_ARG;
+    const AwqWorkspace L = awq_workspace(d_out, d_in, T, group_size);
+    if (workspace_bytes < L.total) return WQ_ERR_INVALID_ARG;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cublasHandle_t h;
+    {
+        std::lock_guard<std::mutex> lk(g_blas_mu);
+        if (!g_blas[st.dev] && cublasCreate(&g_blas[st.dev]) != CUBLAS_STATUS_SUCCESS) return WQ_ERR_CUDA;
+        h = g_blas[st.dev];
+        if (cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS) return WQ_ERR_CUDA;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint16_t* Wp = reinterpret_cast<uint16_t*>(ws + L.wp);
+    uint32_t* qa = reinterpret_cast<uint32_t*>(ws + L.qa);
+    uint16_t* sa = reinterpret_cast<uint16_t*>(ws + L.sa);
+    uint16_t* za = symmetric ? nullptr : reinterpret_cast<uint16_t*>(ws + L.za);
+    uint16_t* Xp = reinterpret_cast<uint16_t*>(ws + L.xp);
+    float* Yref = reinterpret_cast<float*>(ws + L.yref);
+    float* Ya = reinterpret_cast<float*>(ws + L.ya);
+    double* lnm = reinterpret_cast<double*>(ws + L.lnm);
+    double* red = reinterpret_cast<double*>(ws + L.red);
+    double* mean_ln = red + awq_loss_partials();
+    double* loss_buf = losses ? losses : mean_ln + 8;
+    int32_t* best_buf = best ? best : reinterpret_cast<int32_t*>(mean_ln + 32);
+    uint16_t* sbuf = reinterpret_cast<uint16_t*>(ws + L.scal);
+    const uint16_t* W = static_cast<const uint16_t*>(W_bf16);
+    const uint16_t* X = static_cast<const uint16_t*>(X_bf16);
+
+    // reference output Y = X W^T (fp32 accumulation), a plain library GEMM
+    const float one = 1.0f, zero = 0.0f;
+    if (cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, (int)d_out, (int)T, (int)d_in, &one, W, CUDA_R_16BF, (int)d_in, X,
+                     CUDA_R_16BF, (int)d_in, &zero, Yref, CUDA_R_32F, (int)d_out, CUBLAS_COMPUTE_32F,
+                     CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+        return WQ_ERR_CUDA;
+    cudaError_t e = launch_awq_colstats(X, T, d_in, lnm, mean_ln, s);
+    for (int i = 0; e == cudaSuccess && i < kAwqAlphas; ++i) {
+        e = launch_awq_scale_apply(W, d_out, X, T, d_in, lnm, mean_ln, i, nullptr, sbuf, Wp, Xp, st.num_sms, s);
+        if (e == cudaSuccess)
+            e = launch_quantize(Wp, d_out, d_in, group_size, symmetric, qa, sa, za, st.status, st.num_sms, s);
+        if (e == cudaSuccess)
+            e = run_linear(st, Xp, T, qa, sa, za, d_out, d_in, group_size, symmetric, Ya, WQ_OUT_FP32, s);
+        if (e == cudaSuccess) e = launch_awq_loss(Yref, Ya, T * d_out, red, loss_buf + i, s);
+    }
+    if (e == cudaSuccess) e = launch_awq_select(loss_buf, kAwqAlphas, best_buf, s);
+    // the kept alpha: its scales and the RTN artifact of W diag(s) into the caller's buffers
+    if (e == cudaSuccess)
+        e = launch_awq_scale_apply(W, d_out, nullptr, 0, d_in, lnm, mean_ln, 0, best_buf,
+                                   static_cast<uint16_t*>(s_bf16), Wp, nullptr, st.num_sms, s);
+    if (e == cudaSuccess)
+        e = launch_quantize(Wp, d_out, d_in, group_size, symmetric, qweight, static_cast<uint16_t*>(scales_fp16),
+                            static_cast<uint16_t*>(zeros_fp16), st.status, st.num_sms, s);
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+wq_status wq_awq_scale_activations(const void* X_bf16, int64_t T, int64_t d_in, const void* s_bf16, void* Xp_bf16,
+                                    void* stream) {
+    if (!X_bf16 || !s_bf16 || !Xp_bf16 || !aligned(X_bf16, 16) || !aligned(Xp_bf16, 16) || !aligned(s_bf16, 2))
+        return WQ_ERR_INVALID_ARG;
+    if (T < 1 || d_in < 8 || d_in % 8 != 0) return WQ_ERR_INVALID_ARG;
+    DeviceState st;
+    wq_status v = device_state(&st);
+    if (v != WQ_OK) return v;
+    const cudaError_t e = launch_awq_divide(static_cast<const uint16_t*>(X_bf16), T, d_in,
+                                            static_cast<const uint16_t*>(s_bf16), static_cast<uint16_t*>(Xp_bf16),
+                                            st.num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 

@@ -75,6 +75,19 @@ struct GemmArgs {
 
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, const LaunchOptions& opt, cudaStream_t stream);
 
+// AWQ search pieces (awq.cu).
+cudaError_t launch_awq_colstats(const uint16_t* X, int64_t T, int64_t K, double* lnm, double* mean_ln,
+                                cudaStream_t stream);
+cudaError_t launch_awq_scale_apply(const uint16_t* W, int64_t N, const uint16_t* X, int64_t T, int64_t K,
+                                   const double* lnm, const double* mean_ln, int alpha_idx, const int32_t* best,
+                                   uint16_t* s, uint16_t* Wp, uint16_t* Xp, int num_sms, cudaStream_t stream);
+cudaError_t launch_awq_divide(const uint16_t* X, int64_t T, int64_t K, const uint16_t* s, uint16_t* Xp, int num_sms,
+                              cudaStream_t stream);
+cudaError_t launch_awq_loss(const float* Yref, const float* Y, int64_t n, double* part, double* out,
+                            cudaStream_t stream);
+cudaError_t launch_awq_select(const double* losses, int n, int32_t* best, cudaStream_t stream);
+int awq_loss_partials();
+
 cudaError_t launch_bounded_wait_selftest(uint32_t* status, uint32_t limit_us, cudaStream_t stream);
 
 // Driver entry point for tensor-map encoding (resolved once through the runtime).
