@@ -52,12 +52,13 @@ def quant_bytes(N: int, K: int, symmetric: bool, g: int = 128) -> int:
     return N * K * 2 + N * K // 2 + (N * K // g) * per_group
 
 
-def source_digest() -> str:
-    """sha256 over the CUDA sources; DRAM counters taken from an older build do not apply."""
+def source_digest(files) -> str:
+    """sha256 over the CUDA sources a kernel is compiled from; DRAM counters
+    taken from an older version of those sources do not apply."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "w4a16_bit_gemm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
@@ -70,9 +71,9 @@ def kernel_traffic(name: str):
     try:
         with open(path) as f:
             rec = json.load(f)
-    except (OSError, ValueError):
-        return None
-    if rec.get("source_sha256") != source_digest():
+        if rec.get("source_sha256") != source_digest(rec["kernel_sources"]):
+            return None
+    except (OSError, ValueError, KeyError):
         return None
     return rec.get("dram_bytes_per_launch")
 
