@@ -122,6 +122,10 @@ def _load(path: str | None = None):
             lib.wqo_awq_search.restype = i32
             lib.wqo_awq_scales.argtypes = [P, i64, i64, ctypes.c_double, P]
             lib.wqo_awq_scales.restype = None
+            lib.wqo_gptq.argtypes = [P, i64, i64, P, i64, i64, i32, i32, P, P, P, P, P, P, i32]
+            lib.wqo_gptq.restype = i32
+            lib.wqo_gptq_factor.argtypes = [P, i64, i64, i32, P, P, i32]
+            lib.wqo_gptq_factor.restype = ctypes.c_uint32
             lib.wqo_clip_alpha.argtypes = [i32]
             lib.wqo_clip_alpha.restype = ctypes.c_float
             for nm in ("wqo_f32_to_f16_array", "wqo_f32_to_bf16_array", "wqo_f16_to_f32_array"):
@@ -310,6 +314,49 @@ def awq_scales(X_bits: np.ndarray, alpha: float) -> np.ndarray:
     s = np.empty(K, np.uint16)
     _load().wqo_awq_scales(_ptr(X_bits), T, K, float(alpha), _ptr(s))
     return s
+
+
+GPTQ_BLOCK = 128
+
+
+def gptq(W_bits: np.ndarray, X_bits: np.ndarray, group_size: int = 128, symmetric: bool = True,
+         act_order: bool = True, want_factor: bool = False, nthreads: int | None = None):
+    """GPTQ error feedback ([P2] GPTQ chapter and its algorithm; settings
+    default to the page's: 4-bit, group 128, symmetric, act-order on).
+
+    W_bits bf16 [N, K], X_bits bf16 calibration [T, K].  Returns ``(codes
+    [N, K] original column order, scales, zeros or None, perm [K], U [K, K] or
+    None, flags)``; scales/zeros are plain RTN's (static group parameters)."""
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    N, K = W_bits.shape
+    T = X_bits.shape[0]
+    G = K // group_size
+    codes = np.empty((N, K), np.int32)
+    scales = np.empty((N, G), np.uint16)
+    zeros = None if symmetric else np.empty((N, G), np.uint16)
+    perm = np.empty(K, np.int32)
+    U = np.empty((K, K), np.float64) if want_factor else None
+    flags = ctypes.c_uint32(0)
+    rc = _load().wqo_gptq(_ptr(W_bits), N, K, _ptr(X_bits), T, group_size, int(symmetric), int(act_order),
+                          _ptr(codes), _ptr(scales), _ptr(zeros) if zeros is not None else None, _ptr(perm),
+                          _ptr(U) if U is not None else None, ctypes.cast(ctypes.pointer(flags), ctypes.c_void_p),
+                          nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle GPTQ rejected its arguments")
+    return codes, scales, zeros, perm, U, int(flags.value)
+
+
+def gptq_factor(X_bits: np.ndarray, act_order: bool = True, nthreads: int | None = None):
+    """(perm [K], U [K, K], flags): processing order and the upper factor of
+    the inverse of the permuted damped Hessian 2 X^T X."""
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    T, K = X_bits.shape
+    perm = np.empty(K, np.int32)
+    U = np.empty((K, K), np.float64)
+    f = _load().wqo_gptq_factor(_ptr(X_bits), T, K, int(act_order), _ptr(perm), _ptr(U),
+                                nthreads or default_threads())
+    return perm, U, int(f)
 
 
 def pack4(codes: np.ndarray) -> np.ndarray:

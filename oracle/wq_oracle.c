@@ -623,6 +623,273 @@ int wqo_awq_search(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, i
 }
 
 /* ------------------------------------------------------------------------ */
+/* GPTQ: error feedback through the inverse Hessian.                          */
+/* [P2] "Quantization Algorithms" study notes, GPTQ chapter: layer-wise       */
+/* objective ||W X - W_hat X||^2; Hessian H = 2 X X^T with a 1 % dampening of  */
+/* the diagonal; the factor L = Cholesky(H^-1); columns quantized one at a    */
+/* time in blocks of 128 -- err = (w_j - q_j) / L[j][j], the later columns of  */
+/* the block updated with err L[j][.], the columns after the block updated    */
+/* with the block's errors at once; settings W4, group 128, symmetric,        */
+/* act-order on (columns with large |x|^2 first), damp 0.01.                  */
+/* [P1] GPTQ section: one-shot PTQ that corrects the effect of each weight's   */
+/* quantization error on the layer output.                                   */
+/* Readings (the pages leave these open):                                    */
+/*  - X is [T][K] (tokens x input channels), so H = 2 X^T X is K x K;          */
+/*    H[a][b] = 2 sum_t x[t][a] x[t][b], summed in t order;                    */
+/*  - dampening adds d = 0.01 mean(diag H) (diagonal summed in index order)    */
+/*    to every diagonal entry; d = 1 when that mean is 0 (no signal at all);   */
+/*  - act-order: columns are processed by decreasing damped H[j][j], ties in   */
+/*    index order; the permutation applies to H's rows and columns and to W's  */
+/*    columns; without act-order the order is the identity;                   */
+/*  - "Cholesky(H^-1)" is the upper-triangular U with H^-1 = U^T U (the update */
+/*    reads row j of the factor right of the diagonal); H^-1 = Linv^T Linv     */
+/*    with Linv the inverse of the lower Cholesky factor of H;                */
+/*  - quant() is the layer's group-wise quantizer with STATIC parameters: the  */
+/*    scale and zero point of each group of g input channels are plain RTN's   */
+/*    on the original W (the artifact keeps contiguous groups, with or without */
+/*    act-order); a code is clamp(rint(w / s) + z) with w / s the IEEE fp64     */
+/*    quotient of the current weight, and the quantized value is              */
+/*    bf16_rn(s (q - z)), the weight the W4A16 layer multiplies by;           */
+/*  - fp64 throughout, every product rounded before its add or subtract (no    */
+/*    fused multiply-add), sums in ascending index order:                    */
+/*      Cholesky: a[i][j] - l[i][0] l[j][0] - l[i][1] l[j][1] - ... in turn,   */
+/*      then divided by l[j][j] (the diagonal: its square root);              */
+/*      Linv by forward substitution: v = sum_{k=j}^{i-1} l[i][k] Linv[k][j],  */
+/*      Linv[i][j] = -v / l[i][i], Linv[j][j] = 1 / l[j][j];                   */
+/*      H^-1[i][j] = sum_{k >= max(i,j)} Linv[k][i] Linv[k][j];               */
+/*      U by the same Cholesky on H^-1 (U[i][j] = the lower factor's [j][i]);  */
+/*      block tail: acc = sum_{j in block} err_j U[j][k], then w_k -= acc;     */
+/*  - a Cholesky pivot that is not positive and finite (non-finite or          */
+/*    numerically singular input) is replaced by 1 and raises WQO_FLAG_RANGE. */
+/* ------------------------------------------------------------------------ */
+
+#define WQO_GPTQ_BLOCK 128
+
+typedef struct {
+    const uint16_t* X;
+    int64_t T, K;
+    double* H;
+} hess_ctx;
+
+static void hess_rows(void* vctx, int64_t a0, int64_t a1, uint32_t* flags) {
+    hess_ctx* c = (hess_ctx*)vctx;
+    (void)flags;
+    for (int64_t a = a0; a < a1; ++a)
+        for (int64_t b = 0; b < c->K; ++b) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < c->T; ++t)
+                acc += (double)wqo_bf16_to_f32(c->X[t * c->K + a]) * (double)wqo_bf16_to_f32(c->X[t * c->K + b]);
+            c->H[a * c->K + b] = 2.0 * acc;
+        }
+}
+
+/* Lower Cholesky factor of the symmetric A (K x K, row-major), in place in
+ * the lower triangle of L (the strict upper triangle is zeroed). */
+typedef struct {
+    double* L;
+    int64_t K, j;
+} chol_ctx;
+
+static void chol_col_rows(void* vctx, int64_t r0, int64_t r1, uint32_t* flags) {
+    chol_ctx* c = (chol_ctx*)vctx;
+    (void)flags;
+    const int64_t K = c->K, j = c->j;
+    const double ljj = c->L[j * K + j];
+    for (int64_t i = j + 1 + r0; i < j + 1 + r1; ++i) {
+        double v = c->L[i * K + j];
+        for (int64_t k = 0; k < j; ++k) v = v - c->L[i * K + k] * c->L[j * K + k];
+        c->L[i * K + j] = v / ljj;
+    }
+}
+
+static uint32_t cholesky_lower(const double* A, double* L, int64_t K, int nthreads) {
+    uint32_t flags = 0;
+    for (int64_t i = 0; i < K; ++i)
+        for (int64_t j = 0; j < K; ++j) L[i * K + j] = j <= i ? A[i * K + j] : 0.0;
+    for (int64_t j = 0; j < K; ++j) {
+        double d = L[j * K + j];
+        for (int64_t k = 0; k < j; ++k) d = d - L[j * K + k] * L[j * K + k];
+        if (!(d > 0.0) || !isfinite(d)) {
+            d = 1.0;
+            flags |= WQO_FLAG_RANGE;
+        }
+        L[j * K + j] = sqrt(d);
+        chol_ctx c = {L, K, j};
+        if (K - j - 1 > 0) run_rows(chol_col_rows, &c, K - j - 1, (K - j - 1) >= 256 ? nthreads : 1);
+    }
+    return flags;
+}
+
+/* Linv = L^-1 by forward substitution, one column j per unit of work. */
+typedef struct {
+    const double* L;
+    double* Li;
+    int64_t K;
+} trinv_ctx;
+
+static void trinv_cols(void* vctx, int64_t j0, int64_t j1, uint32_t* flags) {
+    trinv_ctx* c = (trinv_ctx*)vctx;
+    (void)flags;
+    const int64_t K = c->K;
+    for (int64_t j = j0; j < j1; ++j) {
+        for (int64_t i = 0; i < j; ++i) c->Li[i * K + j] = 0.0;
+        c->Li[j * K + j] = 1.0 / c->L[j * K + j];
+        for (int64_t i = j + 1; i < K; ++i) {
+            double v = 0.0;
+            for (int64_t k = j; k < i; ++k) v = v + c->L[i * K + k] * c->Li[k * K + j];
+            c->Li[i * K + j] = -v / c->L[i * K + i];
+        }
+    }
+}
+
+/* Hinv[i][j] = sum_{k >= max(i,j)} Linv[k][i] Linv[k][j]. */
+typedef struct {
+    const double* Li;
+    double* Hi;
+    int64_t K;
+} gram_ctx;
+
+static void gram_rows(void* vctx, int64_t i0, int64_t i1, uint32_t* flags) {
+    gram_ctx* c = (gram_ctx*)vctx;
+    (void)flags;
+    const int64_t K = c->K;
+    for (int64_t i = i0; i < i1; ++i)
+        for (int64_t j = 0; j < K; ++j) {
+            double acc = 0.0;
+            for (int64_t k = i > j ? i : j; k < K; ++k) acc = acc + c->Li[k * K + i] * c->Li[k * K + j];
+            c->Hi[i * K + j] = acc;
+        }
+}
+
+/* The factor U (upper, U^T U = H^-1) of the column-permuted damped Hessian
+ * of X; perm[p] is the input channel processed p-th.  U: K x K row-major. */
+uint32_t wqo_gptq_factor(const uint16_t* X, int64_t T, int64_t K, int act_order, int32_t* perm, double* U,
+                         int nthreads) {
+    uint32_t flags = 0;
+    double* H = (double*)malloc(sizeof(double) * (size_t)(K * K));
+    double* Hp = (double*)malloc(sizeof(double) * (size_t)(K * K));
+    double* L = (double*)malloc(sizeof(double) * (size_t)(K * K));
+    hess_ctx hc = {X, T, K, H};
+    run_rows(hess_rows, &hc, K, nthreads);
+    double dsum = 0.0;
+    for (int64_t j = 0; j < K; ++j) dsum += H[j * K + j];
+    double damp = 0.01 * (dsum / (double)K);
+    if (damp == 0.0) damp = 1.0;
+    for (int64_t j = 0; j < K; ++j) H[j * K + j] += damp;
+    /* processing order: insertion sort by decreasing diagonal, stable */
+    for (int64_t j = 0; j < K; ++j) perm[j] = (int32_t)j;
+    if (act_order) {
+        for (int64_t p = 1; p < K; ++p) {
+            int32_t v = perm[p];
+            int64_t q = p;
+#if WQO_MUTANT == 14 /* mistake: act-order ascending */
+            while (q > 0 && H[(int64_t)perm[q - 1] * K + perm[q - 1]] > H[(int64_t)v * K + v]) {
+#else
+            while (q > 0 && H[(int64_t)perm[q - 1] * K + perm[q - 1]] < H[(int64_t)v * K + v]) {
+#endif
+                perm[q] = perm[q - 1];
+                --q;
+            }
+            perm[q] = v;
+        }
+    }
+    for (int64_t a = 0; a < K; ++a)
+        for (int64_t b = 0; b < K; ++b) Hp[a * K + b] = H[(int64_t)perm[a] * K + perm[b]];
+    flags |= cholesky_lower(Hp, L, K, nthreads);
+    trinv_ctx tc = {L, H, K}; /* H now holds Linv */
+    run_rows(trinv_cols, &tc, K, nthreads);
+    gram_ctx gc = {H, Hp, K}; /* Hp now holds H^-1 */
+    run_rows(gram_rows, &gc, K, nthreads);
+    flags |= cholesky_lower(Hp, L, K, nthreads);
+    for (int64_t i = 0; i < K; ++i)
+        for (int64_t j = 0; j < K; ++j) U[i * K + j] = L[j * K + i];
+    free(H);
+    free(Hp);
+    free(L);
+    return flags;
+}
+
+typedef struct {
+    const uint16_t* W;
+    int64_t K, g;
+    const double* U;
+    const int32_t* perm;
+    const uint16_t* scales;
+    const uint16_t* zeros;
+    int qmin, qmax;
+    int32_t* codes;
+} sweep_ctx;
+
+static void sweep_rows(void* vctx, int64_t n0, int64_t n1, uint32_t* flags) {
+    sweep_ctx* c = (sweep_ctx*)vctx;
+    (void)flags;
+    const int64_t K = c->K, G = c->K / c->g;
+    double* w = (double*)malloc(sizeof(double) * (size_t)K);
+    double err[WQO_GPTQ_BLOCK];
+    for (int64_t n = n0; n < n1; ++n) {
+        for (int64_t p = 0; p < K; ++p) w[p] = (double)wqo_bf16_to_f32(c->W[n * K + c->perm[p]]);
+        for (int64_t b0 = 0; b0 < K; b0 += WQO_GPTQ_BLOCK) {
+            const int64_t b1 = b0 + WQO_GPTQ_BLOCK < K ? b0 + WQO_GPTQ_BLOCK : K;
+            for (int64_t j = b0; j < b1; ++j) {
+                const int64_t col = c->perm[j], gi = col / c->g;
+                const uint16_t s16 = c->scales[n * G + gi];
+                const int z = c->zeros ? (int)wqo_f16_to_f32(c->zeros[n * G + gi]) : 0;
+                const double s = (double)wqo_f16_to_f32(s16);
+                int q;
+                if (isnan(w[j])) {
+                    q = z;
+                } else {
+                    double t = rint(w[j] / s) + (double)z;
+                    if (t < (double)c->qmin) t = (double)c->qmin;
+                    if (t > (double)c->qmax) t = (double)c->qmax;
+                    q = (int)t;
+                }
+                c->codes[n * K + col] = q;
+                const double wh = (double)wqo_bf16_to_f32(wqo_dequant_one(s16, q, z));
+#if WQO_MUTANT == 12 /* mistake: error not divided by the pivot */
+                err[j - b0] = w[j] - wh;
+#else
+                err[j - b0] = (w[j] - wh) / c->U[j * K + j];
+#endif
+                for (int64_t k = j + 1; k < b1; ++k) w[k] = w[k] - err[j - b0] * c->U[j * K + k];
+            }
+            for (int64_t k = b1; k < K; ++k) {
+                double acc = 0.0;
+#if WQO_MUTANT == 13 /* mistake: tail update reads the factor transposed */
+                for (int64_t j = b0; j < b1; ++j) acc = acc + err[j - b0] * c->U[k * K + j];
+#else
+                for (int64_t j = b0; j < b1; ++j) acc = acc + err[j - b0] * c->U[j * K + k];
+#endif
+                w[k] = w[k] - acc;
+            }
+        }
+    }
+    free(w);
+}
+
+/* GPTQ of W (bf16 [N][K]) with calibration X (bf16 [T][K]).  Outputs the
+ * codes (original column order), the static RTN scales/zeros, the
+ * processing order perm [K] and optionally U [K][K].  Returns 0, or -1 on
+ * bad arguments; *flags gets WQO_FLAG_* of the RTN pass and the factor. */
+int wqo_gptq(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t T, int64_t g, int symmetric,
+             int act_order, int32_t* codes, uint16_t* scales, uint16_t* zeros, int32_t* perm, double* U_out,
+             uint32_t* flags, int nthreads) {
+    if (!W || !X || !codes || !scales || !perm || N < 1 || K < 1 || T < 1 || g < 1 || K % g != 0) return -1;
+    if (!symmetric && !zeros) return -1;
+    uint32_t f = 0;
+    if (wqo_quantize(W, N, K, g, 4, symmetric, 0, codes, scales, symmetric ? NULL : zeros, &f, nthreads) != 0)
+        return -1;
+    double* U = U_out ? U_out : (double*)malloc(sizeof(double) * (size_t)(K * K));
+    f |= wqo_gptq_factor(X, T, K, act_order, perm, U, nthreads);
+    sweep_ctx sc = {W, K, g, U, perm, scales, symmetric ? NULL : zeros, symmetric ? -8 : 0, symmetric ? 7 : 15,
+                    codes};
+    run_rows(sweep_rows, &sc, N, nthreads);
+    if (!U_out) free(U);
+    if (flags) *flags = f;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Packing (4-bit only): 8 nibbles per uint32, low nibble first.             */
 /* ------------------------------------------------------------------------ */
 

@@ -2,12 +2,14 @@
 in with -DWQO_MUTANT=k) must fail at least one pin, and the real oracle must
 pass the same pins.  This shows the pins constrain every step: statistics,
 scale, zero point, rounding, packing, dequantization, the linear layer and
-the clipping search (error formula and selection) and the AWQ scales."""
+the clipping search (error formula and selection), the AWQ scales and
+GPTQ (pivot division, tail update, processing order)."""
 import pytest
 
 import oracle
 from tests import test_oracle_awq_pins as awq_pins
 from tests import test_oracle_clip_pins as clip_pins
+from tests import test_oracle_gptq_pins as gptq_pins
 from tests import test_oracle_pins as pins
 
 PINS = [
@@ -25,6 +27,9 @@ PINS = [
     clip_pins.test_never_worse_than_rtn,
     awq_pins.test_scales_follow_the_page_formula,
     awq_pins.test_losses_and_choice_recomputed_independently,
+    gptq_pins.test_factor_is_the_upper_cholesky_of_the_damped_inverse_hessian,
+    lambda: gptq_pins.test_codes_match_an_independent_unblocked_sweep(gptq_pins.CASES[0]),
+    gptq_pins.test_obq_two_column_step,
 ]
 
 MUTANTS = {
@@ -38,6 +43,9 @@ MUTANTS = {
     9: "clip search sums absolute errors",
     10: "clip search keeps the largest error",
     11: "AWQ scales inverted",
+    12: "GPTQ error not divided by the pivot",
+    13: "GPTQ tail update reads the factor transposed",
+    14: "GPTQ act-order ascending",
 }
 
 
