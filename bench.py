@@ -352,7 +352,29 @@ def run_ours(args, dist: Dist):
     secondary["awq_search"] = {"shape": "4096x4096", "calib_tokens": T_CAL, "alphas": 11,
                                "ms_per_search": ta * 1e3, "alpha": a_best / 10.0,
                                "loss_vs_rtn": float(a_losses[a_best] / a_losses[0])}
-    del r_awq, ws, Xc
+    del r_awq, ws
+    # GPTQ (fp64 Hessian, inverse factor and error-feedback sweep), the page's
+    # setting: symmetric, group 128, act-order; same calibration activations
+    gws = torch.empty(b.wq_gptq_workspace_bytes(D, D), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        p_g, _ = b.gptq(W, Xc, G128, True, True, workspace=gws)
+    torch.cuda.synchronize()
+    dist.barrier()
+    gsteps = 3
+    ev0.record()
+    for _ in range(gsteps):
+        p_g, _ = b.gptq(W, Xc, G128, True, True, workspace=gws)
+    ev1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    tgq = dist.max(ev0.elapsed_time(ev1) / 1e3) / gsteps
+    p_r = b.quantize_rtn(W, G128, True)
+    Wd64, Xd64 = W.double(), Xc.double()
+    e_g = float((((Wd64 - b.dequantize(p_g).double()) @ Xd64.T) ** 2).sum())
+    e_r = float((((Wd64 - b.dequantize(p_r).double()) @ Xd64.T) ** 2).sum())
+    secondary["gptq"] = {"shape": "4096x4096", "calib_tokens": T_CAL, "symmetric": True, "act_order": True,
+                         "ms_per_layer": tgq * 1e3, "output_sq_error_vs_rtn": e_g / e_r}
+    del gws, p_g, p_r, Wd64, Xd64, Xc
     What = [torch.empty(D, D, dtype=torch.bfloat16, device="cuda") for _ in range(QC)]
 
     def dfn():

@@ -247,6 +247,59 @@ wq_status wq_awq_scale_activations(const void* X_bf16, int64_t T, int64_t d_in, 
                                    void* Xp_bf16, void* stream);
 
 /*
+ * wq_gptq -- GPTQ: group-wise 4-bit quantization with error feedback through
+ * the inverse Hessian of the layer's calibration activations ("Quantization
+ * Algorithms" study notes, GPTQ chapter and its algorithm; "LLM
+ * Quantization: GPTQ, AWQ, SmoothQuant, FP8, KV Cache (7/10)", GPTQ section).
+ * It minimises ||W X - W_hat X||^2 one column at a time, feeding each
+ * column's quantization error into the columns not yet quantized.
+ *
+ * For calibration activations X[T][d_in], in fp64 throughout:
+ *   H = 2 X^T X (d_in x d_in), plus d = 0.01 mean(diag H) on the diagonal
+ *   (d = 1 if that mean is 0);
+ *   processing order: by decreasing H[j][j] with act_order = 1 (ties in
+ *   index order), else the index order;
+ *   U = the upper Cholesky factor of H^-1 (H^-1 = U^T U), H permuted to the
+ *   processing order;
+ *   per row of W, per block of 128 columns in processing order, per column j:
+ *     q_j = clamp(rint(w_j / s) + z) with the group's s and z,
+ *     err_j = (w_j - bf16_rn(s (q_j - z))) / U[j][j],
+ *     w_k -= err_j U[j][k] for the block's later columns k;
+ *   after the block, w_k -= sum_{j in block} err_j U[j][k] for every later k.
+ * Group parameters are static: the scale and zero point of each group are
+ * those wq_quantize_rtn gives for W, so the artifact has the same layout and
+ * feeds wq_dequantize and wq_linear_w4a16 unchanged (the processing order is
+ * internal; no column permutation is stored).  Every product is rounded
+ * before its add (no fused multiply-add) and every sum runs in ascending
+ * index order, so the result is deterministic and defined bit for bit.
+ *
+ *   W_bf16      [d_out][d_in] bf16 weights, input.  16-byte aligned.
+ *   X_bf16      [T][d_in] bf16 calibration activations.  16-byte aligned.
+ *   T           calibration tokens, 1 .. 2^31 - 1.
+ *   group_size, symmetric, qweight, scales_fp16, zeros_fp16: as
+ *               wq_quantize_rtn (the page's setting is symmetric, g = 128).
+ *   act_order   1: columns with large calibration energy first; 0: in order.
+ *   perm        device int32 [d_in] output (the processing order), or NULL.
+ *   workspace   device scratch of wq_gptq_workspace_bytes(d_out, d_in) bytes,
+ *               256-byte aligned, owned by the caller (about
+ *               16 d_in^2 + 9 d_out d_in bytes).
+ * All work is queued on `stream`; the call does not synchronize.
+ * Errors: WQ_ERR_INVALID_ARG as wq_quantize_rtn, plus a bad T or act_order,
+ * or a missing or small workspace; WQ_ERR_CUDA if a launch fails.
+ * Device flags: as wq_quantize_rtn for W; WQ_DEVFLAG_RANGE if a Cholesky
+ * pivot was not positive and finite (non-finite or numerically singular
+ * calibration data; the pivot is then taken as 1 and the result is
+ * unspecified but memory-safe).
+ */
+wq_status wq_gptq(const void* W_bf16, int64_t d_out, int64_t d_in, const void* X_bf16, int64_t T,
+                  int32_t group_size, int32_t symmetric, int32_t act_order, uint32_t* qweight,
+                  void* scales_fp16, void* zeros_fp16, int32_t* perm, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/* Scratch bytes wq_gptq needs (0 for invalid shapes). */
+size_t wq_gptq_workspace_bytes(int64_t d_out, int64_t d_in);
+
+/*
  * wq_get_device_error -- synchronize `stream`, read and clear the device
  * status word of the current device.  *flags receives the WQ_DEVFLAG_* bits
  * (may be NULL).  Returns WQ_OK when no bit was set, otherwise the status of

@@ -28,7 +28,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("wq_quantize_rtn", "wq_quantize_clip_mse", "wq_awq_search", "wq_awq_workspace_bytes",
-              "wq_awq_scale_activations", "wq_dequantize", "wq_linear_w4a16", "wq_linear_workspace_bytes",
+              "wq_awq_scale_activations", "wq_gptq", "wq_gptq_workspace_bytes", "wq_dequantize", "wq_linear_w4a16", "wq_linear_workspace_bytes",
               "wq_get_device_error", "wq_status_string", "wq_abi_version"):
         assert n in names
 
@@ -130,3 +130,22 @@ def test_awq_scale_activations_rejects(lib):
     assert lib.wq_awq_scale_activations(FAKE, 0, 256, FAKE, FAKE, None) == 1
     assert lib.wq_awq_scale_activations(FAKE, 4, 252, FAKE, FAKE, None) == 1
     assert lib.wq_awq_scale_activations(FAKE + 8, 4, 256, FAKE, FAKE, None) == 1
+
+
+@pytest.mark.parametrize("case", [
+    dict(W=None), dict(X=None), dict(X=FAKE + 2), dict(T=0), dict(act=2), dict(ws=None), dict(wsb=64),
+    dict(ws=FAKE + 64), dict(perm=FAKE + 2), dict(zeros=None), dict(g=100),
+])
+def test_gptq_rejects(lib, case):
+    a = dict(W=FAKE, d_out=4, d_in=256, X=FAKE, T=8, g=128, sym=0, act=1, q=FAKE, sc=FAKE, zeros=FAKE, perm=None,
+             ws=FAKE, wsb=1 << 30)
+    a.update(case)
+    st = lib.wq_gptq(a["W"], a["d_out"], a["d_in"], a["X"], a["T"], a["g"], a["sym"], a["act"], a["q"], a["sc"],
+                     a["zeros"], a["perm"], a["ws"], a["wsb"], None)
+    assert st == 1
+
+
+def test_gptq_workspace_query(lib):
+    n = lib.wq_gptq_workspace_bytes(4096, 4096)
+    assert n >= 2 * 4096 * 4096 * 8 + 4096 * 4096 * 8 and n < 2 * 4096 * 4096 * 8 + 4096 * 4096 * 10 + (1 << 24)
+    assert lib.wq_gptq_workspace_bytes(0, 256) == 0

@@ -64,6 +64,10 @@ def _load() -> ctypes.CDLL:
     lib.wq_awq_workspace_bytes.restype = sz
     lib.wq_awq_scale_activations.argtypes = [P, i64, i64, P, P, P]
     lib.wq_awq_scale_activations.restype = ctypes.c_int
+    lib.wq_gptq.argtypes = [P, i64, i64, P, i64, i32, i32, i32, P, P, P, P, P, sz, P]
+    lib.wq_gptq.restype = ctypes.c_int
+    lib.wq_gptq_workspace_bytes.argtypes = [i64, i64]
+    lib.wq_gptq_workspace_bytes.restype = sz
     lib.wq_get_device_error.argtypes = [P, P]
     lib.wq_get_device_error.restype = ctypes.c_int
     lib.wq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
@@ -139,6 +143,16 @@ def wq_awq_workspace_bytes(d_out, d_in, T, group_size) -> int:
 
 def wq_awq_scale_activations(X, T, d_in, s, Xp, stream=None) -> int:
     return lib.wq_awq_scale_activations(_ptr(X), T, d_in, _ptr(s), _ptr(Xp), _stream(stream))
+
+
+def wq_gptq(W, d_out, d_in, X, T, group_size, symmetric, act_order, qweight, scales, zeros, perm, workspace,
+            workspace_bytes, stream=None) -> int:
+    return lib.wq_gptq(_ptr(W), d_out, d_in, _ptr(X), T, group_size, int(symmetric), int(act_order), _ptr(qweight),
+                       _ptr(scales), _ptr(zeros), _ptr(perm), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def wq_gptq_workspace_bytes(d_out, d_in) -> int:
+    return int(lib.wq_gptq_workspace_bytes(d_out, d_in))
 
 
 def wq_linear_workspace_bytes(M, d_out, d_in) -> int:
@@ -254,6 +268,29 @@ def awq_search(W: torch.Tensor, X: torch.Tensor, group_size: int = 128, symmetri
     _check(wq_awq_search(W, d_out, d_in, X, T, group_size, symmetric, out.qweight, out.scales, out.zeros, s, losses,
                          best, workspace, workspace.numel() * workspace.element_size(), stream), "wq_awq_search")
     return AWQResult(out, s, losses, best)
+
+
+def gptq(W: torch.Tensor, X: torch.Tensor, group_size: int = 128, symmetric: bool = True, act_order: bool = True,
+         workspace: torch.Tensor | None = None, stream=None):
+    """GPTQ of bf16 W[d_out, d_in] with calibration activations X[T, d_in]
+    (defaults: the page's symmetric, group 128, act-order).  Returns
+    (PackedLinear, perm) with perm the int32 processing order."""
+    _require_cuda(W, X)
+    if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D bf16 CUDA tensor")
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or not X.is_contiguous() or X.shape[1] != W.shape[1]:
+        raise ValueError("X must be a contiguous [T, d_in] bf16 CUDA tensor")
+    d_out, d_in = W.shape
+    if d_in % group_size != 0:
+        raise ValueError("group_size must divide d_in")
+    out = alloc_packed(d_out, d_in, group_size, symmetric, W.device)
+    perm = torch.empty(d_in, dtype=torch.int32, device=W.device)
+    need = wq_gptq_workspace_bytes(d_out, d_in)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    _check(wq_gptq(W, d_out, d_in, X, X.shape[0], group_size, symmetric, act_order, out.qweight, out.scales,
+                   out.zeros, perm, workspace, workspace.numel() * workspace.element_size(), stream), "wq_gptq")
+    return out, perm
 
 
 def awq_scale_activations(X: torch.Tensor, s: torch.Tensor, out: torch.Tensor | None = None,

@@ -362,6 +362,35 @@ wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const v
     return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 
+size_t wq_gptq_workspace_bytes(int64_t d_out, int64_t d_in) {
+    if (d_out < 1 || d_in < 1) return 0;
+    return gptq_workspace_bytes(d_out, d_in);
+}
+
+wq_status wq_gptq(const void* W_bf16, int64_t d_out, int64_t d_in, const void* X_bf16, int64_t T, int32_t group_size,
+                  int32_t symmetric, int32_t act_order, uint32_t* qweight, void* scales_fp16, void* zeros_fp16,
+                  int32_t* perm, void* workspace, size_t workspace_bytes, void* stream) {
+    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
+    if (v != WQ_OK) return v;
+    if (!W_bf16 || !X_bf16 || !workspace || !aligned(W_bf16, 16) || !aligned(X_bf16, 16) || !aligned(workspace, 256))
+        return WQ_ERR_INVALID_ARG;
+    if (T < 1 || T > (1ll << 31) - 1 || (act_order != 0 && act_order != 1)) return WQ_ERR_INVALID_ARG;
+    if (perm && !aligned(perm, 4)) return WQ_ERR_INVALID_ARG;
+    if (workspace_bytes < gptq_workspace_bytes(d_out, d_in)) return WQ_ERR_INVALID_ARG;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // static group parameters: plain RTN of W (its codes are replaced below)
+    cudaError_t e = launch_quantize(W_bf16, d_out, d_in, group_size, symmetric, qweight,
+                                    static_cast<uint16_t*>(scales_fp16), static_cast<uint16_t*>(zeros_fp16), st.status,
+                                    st.num_sms, s);
+    if (e == cudaSuccess)
+        e = launch_gptq(static_cast<const uint16_t*>(W_bf16), d_out, d_in, static_cast<const uint16_t*>(X_bf16), T,
+                        group_size, symmetric, act_order, qweight, static_cast<const uint16_t*>(scales_fp16),
+                        static_cast<const uint16_t*>(zeros_fp16), perm, workspace, st.status, s);
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
 wq_status wq_awq_scale_activations(const void* X_bf16, int64_t T, int64_t d_in, const void* s_bf16, void* Xp_bf16,
                                     void* stream) {
     if (!X_bf16 || !s_bf16 || !Xp_bf16 || !aligned(X_bf16, 16) || !aligned(Xp_bf16, 16) || !aligned(s_bf16, 2))

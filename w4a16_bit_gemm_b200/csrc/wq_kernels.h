@@ -88,6 +88,12 @@ cudaError_t launch_awq_loss(const float* Yref, const float* Y, int64_t n, double
 cudaError_t launch_awq_select(const double* losses, int n, int32_t* best, cudaStream_t stream);
 int awq_loss_partials();
 
+// GPTQ (gptq.cu): scales/zeros must already hold the RTN parameters of W.
+size_t gptq_workspace_bytes(int64_t N, int64_t K);
+cudaError_t launch_gptq(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t T, int g, int symmetric,
+                        int act_order, uint32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
+                        int32_t* perm_out, void* workspace, uint32_t* status, cudaStream_t stream);
+
 cudaError_t launch_bounded_wait_selftest(uint32_t* status, uint32_t limit_us, cudaStream_t stream);
 
 // Driver entry point for tensor-map encoding (resolved once through the runtime).
