@@ -122,6 +122,10 @@ def _load(path: str | None = None):
             lib.wqo_awq_search.restype = i32
             lib.wqo_awq_scales.argtypes = [P, i64, i64, ctypes.c_double, P]
             lib.wqo_awq_scales.restype = None
+            lib.wqo_pack8.argtypes = [P, i64, i64, P]
+            lib.wqo_pack8.restype = i32
+            lib.wqo_unpack8.argtypes = [P, i64, i64, P]
+            lib.wqo_unpack8.restype = i32
             lib.wqo_gptq.argtypes = [P, i64, i64, P, i64, i64, i32, i32, P, P, P, P, P, P, i32]
             lib.wqo_gptq.restype = i32
             lib.wqo_gptq_factor.argtypes = [P, i64, i64, i32, P, P, i32]
@@ -375,6 +379,32 @@ def unpack4(qweight: np.ndarray, d_in: int, symmetric: bool) -> np.ndarray:
     if _load().wqo_unpack4(_ptr(qweight), d_out, d_in, int(symmetric), _ptr(codes)) != 0:
         raise ValueError("oracle unpack4 rejected its arguments")
     return codes
+
+
+def pack8(codes: np.ndarray) -> np.ndarray:
+    """4 signed 8-bit codes per uint32, low byte first."""
+    codes = np.ascontiguousarray(codes, dtype=np.int32)
+    d_out, d_in = codes.shape
+    q = np.empty((d_out, d_in // 4), np.uint32)
+    if _load().wqo_pack8(_ptr(codes), d_out, d_in, _ptr(q)) != 0:
+        raise ValueError("oracle pack8 rejected its arguments")
+    return q
+
+
+def unpack8(qweight: np.ndarray, d_in: int) -> np.ndarray:
+    qweight = np.ascontiguousarray(qweight, dtype=np.uint32)
+    d_out = qweight.shape[0]
+    codes = np.empty((d_out, d_in), np.int32)
+    if _load().wqo_unpack8(_ptr(qweight), d_out, d_in, _ptr(codes)) != 0:
+        raise ValueError("oracle unpack8 rejected its arguments")
+    return codes
+
+
+def quantize_pack8(W_bits: np.ndarray, group_size: int, nthreads: int | None = None):
+    """Symmetric INT8 ([-127, 127]) quantize + pack: ``(qweight uint32
+    [d_out, d_in/4], scales, flags, codes)``."""
+    codes, scales, _, flags = quantize(W_bits, group_size, 8, True, True, nthreads)
+    return pack8(codes), scales, flags, codes
 
 
 def dequantize(codes: np.ndarray, scales: np.ndarray, zeros, group_size: int,

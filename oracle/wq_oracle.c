@@ -911,6 +911,30 @@ int wqo_pack4(const int32_t* codes, int64_t d_out, int64_t d_in, uint32_t* qweig
     return 0;
 }
 
+/* 8-bit packing (W8A16, [P1] weight-only INT8; [P2] 1.8 symmetric INT8 uses
+ * [-127, 127]): 4 codes per uint32, byte j of word c holds column 4c+j as an
+ * 8-bit two's complement value (bits 8j..8j+7, low byte first). */
+int wqo_pack8(const int32_t* codes, int64_t d_out, int64_t d_in, uint32_t* qweight) {
+    if (!codes || !qweight || d_in % 4 != 0) return -1;
+    for (int64_t r = 0; r < d_out; ++r)
+        for (int64_t c4 = 0; c4 < d_in / 4; ++c4) {
+            uint32_t w = 0;
+            for (int j = 0; j < 4; ++j) w |= ((uint32_t)codes[r * d_in + c4 * 4 + j] & 0xffu) << (8 * j);
+            qweight[r * (d_in / 4) + c4] = w;
+        }
+    return 0;
+}
+
+int wqo_unpack8(const uint32_t* qweight, int64_t d_out, int64_t d_in, int32_t* codes) {
+    if (!codes || !qweight || d_in % 4 != 0) return -1;
+    for (int64_t r = 0; r < d_out; ++r)
+        for (int64_t c = 0; c < d_in; ++c) {
+            int32_t b = (int32_t)((qweight[r * (d_in / 4) + c / 4] >> (8 * (c % 4))) & 0xffu);
+            codes[r * d_in + c] = b >= 128 ? b - 256 : b;
+        }
+    return 0;
+}
+
 /* Inverse of wqo_pack4: symmetric nibbles are read as 4-bit two's complement. */
 int wqo_unpack4(const uint32_t* qweight, int64_t d_out, int64_t d_in, int symmetric,
                 int32_t* codes) {

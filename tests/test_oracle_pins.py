@@ -367,6 +367,29 @@ def test_degenerate_and_nonfinite_groups():
 # Packing layout v1
 # --------------------------------------------------------------------------
 
+def test_pack8_layout_low_byte_first():
+    """W8A16 artifact: 4 codes per word, byte j = column 4c + j, two's complement."""
+    codes = np.array([[1, -1, 127, -127, 0, 5, -2, 64]], np.int32)
+    q = oracle.pack8(codes)
+    assert q.tolist() == [[0x81_7F_FF_01, 0x40_FE_05_00]]
+    assert np.array_equal(oracle.unpack8(q, 8), codes)
+
+
+def test_int8_per_channel_scale_is_amax_over_127():
+    """Per-channel INT8 (group = d_in): s = fp16(amax / 127) per row, codes
+    rint(x / s) in [-127, 127]; the row's largest magnitude maps to +-127."""
+    rng = np.random.default_rng(8)
+    W = bf16_bits(rng.standard_normal((16, 96)).astype(np.float32) * 0.05)
+    qw, sc, flags, codes = oracle.quantize_pack8(W, 96)
+    x = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).float().numpy()
+    amax = np.abs(x).max(axis=1)
+    s_ref = np.array([np.float16(np.float32(a) / np.float32(127.0)) for a in amax])
+    assert np.array_equal(sc[:, 0], s_ref.view(np.uint16)) and flags == 0
+    s32 = s_ref.astype(np.float32)[:, None]
+    assert np.array_equal(codes, np.clip(np.rint((x / s32).astype(np.float32)), -127, 127).astype(np.int32))
+    assert np.all(np.abs(codes).max(axis=1) == 127)
+    assert np.array_equal(oracle.unpack8(qw, 96), codes)
+
 def test_pack_layout_low_nibble_first():
     codes = np.array([[0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15]], np.int32)
     q = oracle.pack4(codes)
