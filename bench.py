@@ -395,6 +395,45 @@ def run_ours(args, dist: Dist):
         r["frac_of_measured_hbm"] = r["GBps"] / hbm
         secondary["gemv"].append(r)
 
+    # ---------------- W8A16 (symmetric INT8, per-channel) ----------------
+    # decode GEMV M=1 and M=16 on the 4096 x 4096 projection, 64 distinct copies
+    # per sweep (1.07 GB > L2), then the prefill GEMM at M=2048 on 8192 x 8192
+    secondary["w8a16"] = []
+    W8 = syn.case_weight(syn.ATTN, 0, "cuda")
+    p8 = b.quantize_w8(W8)
+    del W8
+    p8s = [b.PackedLinearW8(p8.qweight.clone(), p8.scales.clone(), D, D, D) for _ in range(NCOPY)]
+    for M in (1, 16):
+        X8 = syn.case_activations(syn.ATTN, 0, M, "cuda")
+        Y8 = [torch.empty(M, D, dtype=torch.bfloat16, device="cuda") for _ in range(NCOPY)]
+
+        def w8fn():
+            for i in range(NCOPY):
+                b.linear_w8a16(X8, p8s[i], out=Y8[i])
+        g8 = capture(w8fn)
+        t8 = dist.max(timed_graph(g8, ssteps, 3, dist)) / (ssteps * NCOPY)
+        nb8 = D * D + 2 * D + 2 * M * (D + D)
+        secondary["w8a16"].append({"shape": "4096x4096", "M": M, "group": "per-channel", "us_per_launch": t8 * 1e6,
+                                   "GBps": nb8 / t8 / 1e9, "bytes_per_launch": nb8,
+                                   "frac_of_measured_hbm": nb8 / t8 / 1e9 / hbm})
+        del g8, Y8
+    del p8s, p8
+    torch.cuda.empty_cache()
+    cc = syn.PREFILL.cases[0]
+    Wg8 = syn.case_weight(syn.PREFILL, 0, "cuda")
+    pg8 = b.quantize_w8(Wg8, G128)
+    del Wg8
+    Xg8 = syn.case_activations(syn.PREFILL, 0, 2048, "cuda")
+    Yg8 = torch.empty(2048, cc.d_out, dtype=torch.bfloat16, device="cuda")
+    gg8 = capture(lambda: b.linear_w8a16(Xg8, pg8, out=Yg8))
+    tg8 = dist.max(timed_graph(gg8, 20, 3, dist)) / 20
+    fl8 = 2.0 * 2048 * cc.d_out * cc.d_in
+    secondary["w8a16"].append({"shape": f"{cc.d_out}x{cc.d_in}", "M": 2048, "group": 128,
+                               "ms_per_launch": tg8 * 1e3, "TFLOPs": fl8 / tg8 / 1e12,
+                               "frac_of_measured_bf16": fl8 / tg8 / 1e12 / tf_burst})
+    del gg8, pg8, Xg8, Yg8
+    torch.cuda.empty_cache()
+
     # ---------------- GEMM TFLOP/s (config 4) ----------------
     secondary["gemm"] = []
     for (ci, M) in ((0, 512), (0, 2048), (1, 8192)):

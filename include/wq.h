@@ -247,6 +247,41 @@ wq_status wq_awq_scale_activations(const void* X_bf16, int64_t T, int64_t d_in, 
                                    void* Xp_bf16, void* stream);
 
 /*
+ * W8A16: symmetric INT8 weights with bf16 activations ("LLM Quantization:
+ * GPTQ, AWQ, SmoothQuant, FP8, KV Cache (7/10)", "Which tensor is quantized":
+ * weight-only INT4 / INT8 with 16-bit activations; Granularity: per-channel
+ * is one group spanning d_in; "Quantization Algorithms" study notes 1.8:
+ * symmetric INT8 uses [-127, 127]).
+ *
+ * Artifact (layout "w8 v1"):
+ *   qweight  uint32 [d_out][d_in/4]: byte j of word c = code of column 4c+j,
+ *            8-bit two's complement in [-127, 127], low byte first.
+ *   scales   fp16 [d_out][d_in/group_size].  No zero points.
+ * group_size: a multiple of 32 that divides d_in (d_in itself = per-channel);
+ * d_in must be a multiple of 32.
+ *
+ * wq_quantize_w8 -- s = fp16_rn(fl32(amax / 127)) per group, the maximum
+ * over the group's finite and infinite values (NaN skipped); a zero scale
+ * becomes 1; an fp16 overflow saturates to 65504 (WQ_DEVFLAG_RANGE);
+ * q = clamp(rint(fl32(x / s)), -127, 127), NaN coded as 0 (non-finite input:
+ * WQ_DEVFLAG_NONFINITE).  W_bf16 16-byte aligned.
+ * wq_dequantize_w8 -- x_hat = bf16_rn(s q) (exact fp32 product, one
+ * rounding).  W_hat_bf16 [d_out][d_in], 16-byte aligned.
+ * wq_linear_w8a16 -- Y[M][d_out] = X[M][d_in] . x_hat^T with fp32
+ * accumulation; M <= 16 runs a tensor-core GEMV, larger M the tcgen05 GEMM.
+ * X and Y 16-byte aligned; y_dtype as wq_linear_w4a16.
+ * Errors: WQ_ERR_INVALID_ARG for null or misaligned pointers and shapes
+ * outside the rules above; WQ_ERR_CUDA if a launch fails.
+ */
+wq_status wq_quantize_w8(const void* W_bf16, int64_t d_out, int64_t d_in, int32_t group_size,
+                         uint32_t* qweight, void* scales_fp16, void* stream);
+wq_status wq_dequantize_w8(const uint32_t* qweight, const void* scales_fp16, int64_t d_out,
+                           int64_t d_in, int32_t group_size, void* W_hat_bf16, void* stream);
+wq_status wq_linear_w8a16(const void* X_bf16, int64_t M, const uint32_t* qweight,
+                          const void* scales_fp16, int64_t d_out, int64_t d_in, int32_t group_size,
+                          void* Y, int32_t y_dtype, void* stream);
+
+/*
  * wq_gptq -- GPTQ: group-wise 4-bit quantization with error feedback through
  * the inverse Hessian of the layer's calibration activations ("Quantization
  * Algorithms" study notes, GPTQ chapter and its algorithm; "LLM

@@ -28,7 +28,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("wq_quantize_rtn", "wq_quantize_clip_mse", "wq_awq_search", "wq_awq_workspace_bytes",
-              "wq_awq_scale_activations", "wq_gptq", "wq_gptq_workspace_bytes", "wq_dequantize", "wq_linear_w4a16", "wq_linear_workspace_bytes",
+              "wq_awq_scale_activations", "wq_gptq", "wq_gptq_workspace_bytes", "wq_quantize_w8",
+              "wq_dequantize_w8", "wq_linear_w8a16", "wq_dequantize", "wq_linear_w4a16", "wq_linear_workspace_bytes",
               "wq_get_device_error", "wq_status_string", "wq_abi_version"):
         assert n in names
 
@@ -149,3 +150,21 @@ def test_gptq_workspace_query(lib):
     n = lib.wq_gptq_workspace_bytes(4096, 4096)
     assert n >= 2 * 4096 * 4096 * 8 + 4096 * 4096 * 8 and n < 2 * 4096 * 4096 * 8 + 4096 * 4096 * 10 + (1 << 24)
     assert lib.wq_gptq_workspace_bytes(0, 256) == 0
+
+
+@pytest.mark.parametrize("case", [
+    dict(W=None), dict(W=FAKE + 8), dict(q=FAKE + 4), dict(s=None), dict(d_in=1000, g=1000), dict(g=48),
+    dict(g=16, d_in=256), dict(d_in=96, g=64), dict(d_out=0),
+])
+def test_w8_quantize_rejects(lib, case):
+    a = dict(W=FAKE, d_out=4, d_in=256, g=128, q=FAKE, s=FAKE)
+    a.update(case)
+    assert lib.wq_quantize_w8(a["W"], a["d_out"], a["d_in"], a["g"], a["q"], a["s"], None) == 1
+
+
+def test_w8_linear_and_dequant_reject(lib):
+    assert lib.wq_linear_w8a16(FAKE, 0, FAKE, FAKE, 64, 256, 256, FAKE, 0, None) == 1
+    assert lib.wq_linear_w8a16(FAKE + 8, 1, FAKE, FAKE, 64, 256, 256, FAKE, 0, None) == 1
+    assert lib.wq_linear_w8a16(FAKE, 1, FAKE, FAKE, 64, 256, 256, FAKE, 3, None) == 1
+    assert lib.wq_dequantize_w8(FAKE, FAKE, 4, 256, 128, None, None) == 1
+    assert lib.wq_dequantize_w8(FAKE, None, 4, 256, 128, FAKE, None) == 1

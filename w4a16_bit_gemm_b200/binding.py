@@ -64,6 +64,12 @@ def _load() -> ctypes.CDLL:
     lib.wq_awq_workspace_bytes.restype = sz
     lib.wq_awq_scale_activations.argtypes = [P, i64, i64, P, P, P]
     lib.wq_awq_scale_activations.restype = ctypes.c_int
+    lib.wq_quantize_w8.argtypes = [P, i64, i64, i32, P, P, P]
+    lib.wq_quantize_w8.restype = ctypes.c_int
+    lib.wq_dequantize_w8.argtypes = [P, P, i64, i64, i32, P, P]
+    lib.wq_dequantize_w8.restype = ctypes.c_int
+    lib.wq_linear_w8a16.argtypes = [P, i64, P, P, i64, i64, i32, P, i32, P]
+    lib.wq_linear_w8a16.restype = ctypes.c_int
     lib.wq_gptq.argtypes = [P, i64, i64, P, i64, i32, i32, i32, P, P, P, P, P, sz, P]
     lib.wq_gptq.restype = ctypes.c_int
     lib.wq_gptq_workspace_bytes.argtypes = [i64, i64]
@@ -143,6 +149,19 @@ def wq_awq_workspace_bytes(d_out, d_in, T, group_size) -> int:
 
 def wq_awq_scale_activations(X, T, d_in, s, Xp, stream=None) -> int:
     return lib.wq_awq_scale_activations(_ptr(X), T, d_in, _ptr(s), _ptr(Xp), _stream(stream))
+
+
+def wq_quantize_w8(W, d_out, d_in, group_size, qweight, scales, stream=None) -> int:
+    return lib.wq_quantize_w8(_ptr(W), d_out, d_in, group_size, _ptr(qweight), _ptr(scales), _stream(stream))
+
+
+def wq_dequantize_w8(qweight, scales, d_out, d_in, group_size, W_hat, stream=None) -> int:
+    return lib.wq_dequantize_w8(_ptr(qweight), _ptr(scales), d_out, d_in, group_size, _ptr(W_hat), _stream(stream))
+
+
+def wq_linear_w8a16(X, M, qweight, scales, d_out, d_in, group_size, Y, y_dtype, stream=None) -> int:
+    return lib.wq_linear_w8a16(_ptr(X), M, _ptr(qweight), _ptr(scales), d_out, d_in, group_size, _ptr(Y), y_dtype,
+                               _stream(stream))
 
 
 def wq_gptq(W, d_out, d_in, X, T, group_size, symmetric, act_order, qweight, scales, zeros, perm, workspace,
@@ -230,6 +249,61 @@ def quantize_clip_mse(W: torch.Tensor, group_size: int = 128, symmetric: bool = 
         out = alloc_packed(d_out, d_in, group_size, symmetric, W.device)
     _check(wq_quantize_clip_mse(W, d_out, d_in, group_size, symmetric, out.qweight, out.scales, out.zeros, stream),
            "wq_quantize_clip_mse")
+    return out
+
+
+class PackedLinearW8:
+    """Symmetric INT8 artifact (layout w8 v1) of one weight matrix W[d_out, d_in]."""
+
+    def __init__(self, qweight, scales, d_out, d_in, group_size):
+        self.qweight = qweight
+        self.scales = scales
+        self.d_out = d_out
+        self.d_in = d_in
+        self.group_size = group_size
+
+    def nbytes(self) -> int:
+        return self.qweight.numel() * 4 + self.scales.numel() * 2
+
+
+def quantize_w8(W: torch.Tensor, group_size: int | None = None, out: PackedLinearW8 | None = None,
+                stream=None) -> PackedLinearW8:
+    """Symmetric INT8 quantization of bf16 W[d_out, d_in]; group_size None or
+    d_in = per-channel (one scale per output row)."""
+    _require_cuda(W)
+    if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D bf16 CUDA tensor")
+    d_out, d_in = W.shape
+    g = d_in if group_size is None else group_size
+    if out is None:
+        if d_in % g != 0:
+            raise ValueError("group_size must divide d_in")
+        out = PackedLinearW8(torch.empty(d_out, d_in // 4, dtype=torch.int32, device=W.device),
+                             torch.empty(d_out, d_in // g, dtype=torch.float16, device=W.device), d_out, d_in, g)
+    _check(wq_quantize_w8(W, d_out, d_in, g, out.qweight, out.scales, stream), "wq_quantize_w8")
+    return out
+
+
+def dequantize_w8(p: PackedLinearW8, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _require_cuda(p.qweight)
+    if out is None:
+        out = torch.empty(p.d_out, p.d_in, dtype=torch.bfloat16, device=p.qweight.device)
+    _check(wq_dequantize_w8(p.qweight, p.scales, p.d_out, p.d_in, p.group_size, out, stream), "wq_dequantize_w8")
+    return out
+
+
+def linear_w8a16(X: torch.Tensor, p: PackedLinearW8, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """Y[M, d_out] = X[M, d_in] . x_hat^T with fp32 accumulation (INT8 weights)."""
+    _require_cuda(X, p.qweight)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or not X.is_contiguous() or X.shape[1] != p.d_in:
+        raise ValueError("X must be a contiguous [M, d_in] bf16 CUDA tensor")
+    y_dtype = WQ_OUT_FP32 if out_dtype == torch.float32 else WQ_OUT_BF16
+    if out is None:
+        out = torch.empty(X.shape[0], p.d_out, dtype=torch.float32 if y_dtype == WQ_OUT_FP32 else torch.bfloat16,
+                          device=X.device)
+    _check(wq_linear_w8a16(X, X.shape[0], p.qweight, p.scales, p.d_out, p.d_in, p.group_size, out, y_dtype, stream),
+           "wq_linear_w8a16")
     return out
 
 

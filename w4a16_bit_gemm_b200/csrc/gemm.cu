@@ -24,6 +24,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "w8_device.cuh"
 #include "wq_device.cuh"
 #include "wq_kernels.h"
 #include "wq_tcgen05.cuh"
@@ -33,16 +34,17 @@ namespace {
 
 constexpr int kBN = 256;        // output channels per tile (MMA N)
 constexpr int kBK = 64;         // k per stage (one 128-byte swizzle atom of bf16)
-constexpr int kS1 = 4;          // X / packed-W ring depth
 constexpr int kS2 = 2;          // dequantized-W ring depth
 constexpr int kGemmThreads = 320;
 constexpr int kProducerWarp0 = 2;
 constexpr int kNumProducerWarps = 8;
 
-template <int MSUB>
+template <int MSUB, int BITS>
 struct GemmSmem {
+    // X / packed-W ring depth: 4, or 3 when 8-bit tiles would not fit
+    static constexpr int kS1 = (BITS == 8 && MSUB == 2) ? 3 : 4;
     static constexpr int kATile = 128 * MSUB * kBK * 2;  // bytes
-    static constexpr int kWqTile = kBN * kBK / 2;        // packed bytes
+    static constexpr int kWqTile = kBN * kBK * BITS / 8; // packed bytes
     static constexpr int kBTile = kBN * kBK * 2;
     static constexpr int kStage1 = kATile + kWqTile;
     static constexpr int kOffA = 0;                           // S1 x A tiles
@@ -53,11 +55,12 @@ struct GemmSmem {
     static constexpr int kAlloc = kBytes + 1024;              // + alignment slack
 };
 
-template <int MSUB>
+template <int MSUB, int BITS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_w4a16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_wq,
                               const GemmArgs a) {
-    using SL = GemmSmem<MSUB>;
+    using SL = GemmSmem<MSUB, BITS>;
+    constexpr int kS1 = SL::kS1;
     extern __shared__ uint8_t smem_raw[];
     // the dynamic shared-memory base is only guaranteed 16-byte alignment; the
     // 128-byte swizzle atoms need 1024 (the launch adds 1024 bytes of slack)
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                 for (int ms = 0; ms < MSUB; ++ms)
                     tma_load_2d(As + ms * (128 * kBK * 2), &tmap_x, &full1[s], kb * kBK, m0 + 128 * ms);
-                tma_load_2d(smem + SL::kOffWq + s * SL::kWqTile, &tmap_wq, &full1[s], kb * (kBK / 8), n0);
+                tma_load_2d(smem + SL::kOffWq + s * SL::kWqTile, &tmap_wq, &full1[s], kb * (kBK * BITS / 32), n0);
                 ++issued;
             }
             // drain: wait until the last load into every stage has landed
@@ -159,54 +162,92 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int n = n0 + i;
         const bool nvalid = n < a.N;
         const bool sym = a.symmetric != 0;
-        const int kw = a.K / 8;  // packed words per row
+        const int kw = a.K * BITS / 32;  // packed words per row
         for (int kb = 0; kb < nkb; ++kb) {
             const int s1 = kb % kS1, s2 = kb % kS2;
             if (__any_sync(0xffffffffu, *(volatile int*)abort_flag != 0)) break;
             // group constants for the two 32-k halves of this k block
             const int kbase = kb * kBK;
             const int gA = kbase / a.g, gB = (kbase + 32) / a.g;
-            GroupConsts cA, cB;
-            if (nvalid) {
-                const int64_t ia = (int64_t)n * a.G + gA;
-                cA = make_group_consts(a.scales[ia], sym ? 0 : (int)__half2float(__ushort_as_half(a.zeros[ia])), sym);
-                if (gB != gA && kbase + 32 < a.K) {
-                    const int64_t ib = (int64_t)n * a.G + gB;
-                    cB = make_group_consts(a.scales[ib], sym ? 0 : (int)__half2float(__ushort_as_half(a.zeros[ib])),
-                                           sym);
+            uint8_t* brow = smem + SL::kOffB + s2 * SL::kBTile + i * 128;
+            if constexpr (BITS == 4) {
+                GroupConsts cA, cB;
+                if (nvalid) {
+                    const int64_t ia = (int64_t)n * a.G + gA;
+                    cA = make_group_consts(a.scales[ia], sym ? 0 : (int)__half2float(__ushort_as_half(a.zeros[ia])), sym);
+                    if (gB != gA && kbase + 32 < a.K) {
+                        const int64_t ib = (int64_t)n * a.G + gB;
+                        cB = make_group_consts(a.scales[ib], sym ? 0 : (int)__half2float(__ushort_as_half(a.zeros[ib])),
+                                               sym);
+                    } else {
+                        cB = cA;
+                    }
                 } else {
+                    cA = make_group_consts(0x3c00u, 0, sym);
                     cB = cA;
                 }
-            } else {
-                cA = make_group_consts(0x3c00u, 0, sym);
-                cB = cA;
-            }
-            bool ready = mbar_wait(&full1[s1], (uint32_t)(kb / kS1) & 1u, a.status);
-            if (ready && kb >= kS2) ready = mbar_wait(&empty2[s2], (uint32_t)((kb / kS2) - 1) & 1u, a.status);
-            if (!__all_sync(0xffffffffu, ready)) {  // warp-uniform give-up
-                if (lane == 0) atomicExch(abort_flag, 1);
-                break;
-            }
-            // packed row i: 32 bytes, SWIZZLE_32B (16-byte half h stored at h ^ ((i >> 2) & 1))
-            const uint8_t* wq = smem + SL::kOffWq + s1 * SL::kWqTile + i * 32;
-            const int sw = (i >> 2) & 1;
-            const uint4 h0 = *reinterpret_cast<const uint4*>(wq + ((0 ^ sw) << 4));
-            const uint4 h1 = *reinterpret_cast<const uint4*>(wq + ((1 ^ sw) << 4));
-            const uint32_t words[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty1[s1]);  // packed tile no longer needed by this warp
-            uint8_t* brow = smem + SL::kOffB + s2 * SL::kBTile + i * 128;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint32_t o[4];
-                const bool kval = nvalid && (kb * (kBK / 8) + j) < kw;
-                if (kval) {
-                    dequant_word_natural(words[j], j < 4 ? cA : cB, o);
-                } else {
-                    o[0] = o[1] = o[2] = o[3] = 0u;
+                bool ready = mbar_wait(&full1[s1], (uint32_t)(kb / kS1) & 1u, a.status);
+                if (ready && kb >= kS2) ready = mbar_wait(&empty2[s2], (uint32_t)((kb / kS2) - 1) & 1u, a.status);
+                if (!__all_sync(0xffffffffu, ready)) {  // warp-uniform give-up
+                    if (lane == 0) atomicExch(abort_flag, 1);
+                    break;
                 }
-                // 16-byte chunk j of a 128-byte row, swizzled by row % 8
-                *reinterpret_cast<uint4*>(brow + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                // packed row i: 32 bytes, SWIZZLE_32B (16-byte half h stored at h ^ ((i >> 2) & 1))
+                const uint8_t* wq = smem + SL::kOffWq + s1 * SL::kWqTile + i * 32;
+                const int sw = (i >> 2) & 1;
+                const uint4 h0 = *reinterpret_cast<const uint4*>(wq + ((0 ^ sw) << 4));
+                const uint4 h1 = *reinterpret_cast<const uint4*>(wq + ((1 ^ sw) << 4));
+                const uint32_t words[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty1[s1]);  // packed tile no longer needed by this warp
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t o[4];
+                    const bool kval = nvalid && (kb * (kBK / 8) + j) < kw;
+                    if (kval) {
+                        dequant_word_natural(words[j], j < 4 ? cA : cB, o);
+                    } else {
+                        o[0] = o[1] = o[2] = o[3] = 0u;
+                    }
+                    // 16-byte chunk j of a 128-byte row, swizzled by row % 8
+                    *reinterpret_cast<uint4*>(brow + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            } else {
+                float sA = 0.0f, sB = 0.0f;  // symmetric INT8: scales only
+                if (nvalid) {
+                    sA = __half2float(__ushort_as_half(a.scales[(int64_t)n * a.G + gA]));
+                    sB = (gB != gA && kbase + 32 < a.K) ? __half2float(__ushort_as_half(a.scales[(int64_t)n * a.G + gB]))
+                                                         : sA;
+                }
+                bool ready = mbar_wait(&full1[s1], (uint32_t)(kb / kS1) & 1u, a.status);
+                if (ready && kb >= kS2) ready = mbar_wait(&empty2[s2], (uint32_t)((kb / kS2) - 1) & 1u, a.status);
+                if (!__all_sync(0xffffffffu, ready)) {  // warp-uniform give-up
+                    if (lane == 0) atomicExch(abort_flag, 1);
+                    break;
+                }
+                // packed row i: 64 bytes, SWIZZLE_64B (16-byte chunk h stored at h ^ ((i >> 1) & 3))
+                const uint8_t* wq = smem + SL::kOffWq + s1 * SL::kWqTile + i * 64;
+                const int sw = (i >> 1) & 3;
+                uint32_t words[16];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(wq + ((h ^ sw) << 4));
+                    words[4 * h] = v.x;
+                    words[4 * h + 1] = v.y;
+                    words[4 * h + 2] = v.z;
+                    words[4 * h + 3] = v.w;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty1[s1]);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t o[4] = {0u, 0u, 0u, 0u};
+                    if (nvalid && (kb * (kBK / 4) + 2 * j) < kw) {
+                        dequant_word_w8(words[2 * j], j < 4 ? sA : sB, o[0], o[1]);
+                        dequant_word_w8(words[2 * j + 1], j < 4 ? sA : sB, o[2], o[3]);
+                    }
+                    *reinterpret_cast<uint4*>(brow + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
             }
             fence_proxy_async_smem();  // make the generic-proxy stores visible to the tensor core
             __syncwarp();
@@ -278,16 +319,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_gemm(const GemmArgs& a, int num_sms, const LaunchOptions& opt, cudaStream_t stream) {
+namespace {
+
+template <int BITS>
+cudaError_t launch_gemm_bits(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     const int n_tiles = (a.N + kBN - 1) / kBN;
     const int m_tiles256 = (a.M + 255) / 256;
     const bool use2 = (int64_t)m_tiles256 * n_tiles >= num_sms;
+    constexpr int kWordsPerRowStage = kBK * BITS / 32;
     CUtensorMap tx, tw;
     CUresult cr = encode_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.X, (uint64_t)a.K, (uint64_t)a.M,
                                        (uint64_t)a.K * 2, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    cr = encode_tensor_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.qweight, (uint64_t)(a.K / 8), (uint64_t)a.N,
-                              (uint64_t)(a.K / 2), kBK / 8, kBN, CU_TENSOR_MAP_SWIZZLE_32B);
+    cr = encode_tensor_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.qweight, (uint64_t)a.K * BITS / 32,
+                              (uint64_t)a.N, (uint64_t)a.K * BITS / 8, kWordsPerRowStage, kBN,
+                              BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B);
     if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
     cudaLaunchConfig_t cfg = {};
@@ -298,21 +344,33 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, const LaunchOptions& opt
     attr[0].val.programmaticStreamSerializationAllowed = 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    (void)opt;
     if (use2) {
-        auto kern = gemm_w4a16_tcgen05_kernel<2>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem<2>::kAlloc);
+        auto kern = gemm_w4a16_tcgen05_kernel<2, BITS>;
+        constexpr int bytes = GemmSmem<2, BITS>::kAlloc;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) return e;
         cfg.gridDim = dim3(m_tiles256 * n_tiles);
-        cfg.dynamicSmemBytes = GemmSmem<2>::kAlloc;
+        cfg.dynamicSmemBytes = bytes;
         return cudaLaunchKernelEx(&cfg, kern, tx, tw, a);
     }
-    auto kern = gemm_w4a16_tcgen05_kernel<1>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem<1>::kAlloc);
+    auto kern = gemm_w4a16_tcgen05_kernel<1, BITS>;
+    constexpr int bytes = GemmSmem<1, BITS>::kAlloc;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3(((a.M + 127) / 128) * n_tiles);
-    cfg.dynamicSmemBytes = GemmSmem<1>::kAlloc;
+    cfg.dynamicSmemBytes = bytes;
     return cudaLaunchKernelEx(&cfg, kern, tx, tw, a);
+}
+
+static_assert(GemmSmem<2, 4>::kAlloc <= 227 * 1024, "4-bit GEMM shared memory");
+static_assert(GemmSmem<2, 8>::kAlloc <= 227 * 1024, "8-bit GEMM shared memory");
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& a, int num_sms, const LaunchOptions& opt, cudaStream_t stream) {
+    (void)opt;
+    if (a.bits == 8) return launch_gemm_bits<8>(a, num_sms, stream);
+    return launch_gemm_bits<4>(a, num_sms, stream);
 }
 
 }  // namespace wq

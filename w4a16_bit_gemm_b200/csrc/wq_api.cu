@@ -232,6 +232,7 @@ cudaError_t run_linear(const DeviceState& st, const void* X_bf16, int64_t M, con
     a.G = (int)(d_in / group_size);
     a.symmetric = symmetric;
     a.y_fp32 = y_dtype == WQ_OUT_FP32;
+    a.bits = 4;
     return launch_gemm(a, st.num_sms, opt, s);
 }
 
@@ -359,6 +360,95 @@ wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const v
     if (e == cudaSuccess)
         e = launch_quantize(Wp, d_out, d_in, group_size, symmetric, qweight, static_cast<uint16_t*>(scales_fp16),
                             static_cast<uint16_t*>(zeros_fp16), st.status, st.num_sms, s);
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// W8A16
+// ---------------------------------------------------------------------------
+
+namespace {
+
+wq_status check_w8_artifact(const void* qweight, const void* scales, int64_t d_out, int64_t d_in, int32_t g) {
+    if (!qweight || !scales) return WQ_ERR_INVALID_ARG;
+    if (d_out < 1 || d_in < 1 || d_out > (1ll << 31) - 1 || d_in > (1ll << 31) - 1) return WQ_ERR_INVALID_ARG;
+    if (d_in % 32 != 0 || g < 32 || g % 32 != 0 || d_in % g != 0) return WQ_ERR_INVALID_ARG;
+    if (!aligned(qweight, 16) || !aligned(scales, 2)) return WQ_ERR_INVALID_ARG;
+    return WQ_OK;
+}
+
+}  // namespace
+
+wq_status wq_quantize_w8(const void* W_bf16, int64_t d_out, int64_t d_in, int32_t group_size, uint32_t* qweight,
+                         void* scales_fp16, void* stream) {
+    wq_status v = check_w8_artifact(qweight, scales_fp16, d_out, d_in, group_size);
+    if (v != WQ_OK) return v;
+    if (!W_bf16 || !aligned(W_bf16, 16)) return WQ_ERR_INVALID_ARG;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    const cudaError_t e = launch_quantize_w8(W_bf16, d_out, d_in, group_size, qweight,
+                                             static_cast<uint16_t*>(scales_fp16), st.status, st.num_sms,
+                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+wq_status wq_dequantize_w8(const uint32_t* qweight, const void* scales_fp16, int64_t d_out, int64_t d_in,
+                           int32_t group_size, void* W_hat_bf16, void* stream) {
+    wq_status v = check_w8_artifact(qweight, scales_fp16, d_out, d_in, group_size);
+    if (v != WQ_OK) return v;
+    if (!W_hat_bf16 || !aligned(W_hat_bf16, 16)) return WQ_ERR_INVALID_ARG;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    const cudaError_t e = launch_dequantize_w8(qweight, static_cast<const uint16_t*>(scales_fp16), d_out, d_in,
+                                               group_size, W_hat_bf16, st.num_sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
+}
+
+wq_status wq_linear_w8a16(const void* X_bf16, int64_t M, const uint32_t* qweight, const void* scales_fp16,
+                          int64_t d_out, int64_t d_in, int32_t group_size, void* Y, int32_t y_dtype, void* stream) {
+    wq_status v = check_w8_artifact(qweight, scales_fp16, d_out, d_in, group_size);
+    if (v != WQ_OK) return v;
+    if (!X_bf16 || !Y || !aligned(X_bf16, 16) || !aligned(Y, 16)) return WQ_ERR_INVALID_ARG;
+    if (M < 1 || M > (1ll << 31) - 1) return WQ_ERR_INVALID_ARG;
+    if (y_dtype != WQ_OUT_BF16 && y_dtype != WQ_OUT_FP32) return WQ_ERR_INVALID_ARG;
+    DeviceState st;
+    if ((v = device_state(&st)) != WQ_OK) return v;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (M <= 16) {
+        W8Args a = {};
+        a.X = X_bf16;
+        a.qweight = qweight;
+        a.scales = static_cast<const uint16_t*>(scales_fp16);
+        a.Y = Y;
+        a.status = st.status;
+        a.N = d_out;
+        a.K = d_in;
+        a.G = d_in / group_size;
+        a.M = (int)M;
+        a.g = group_size;
+        a.y_fp32 = y_dtype == WQ_OUT_FP32;
+        e = launch_gemv_w8a16(a, s);
+    } else {
+        GemmArgs a = {};
+        a.X = X_bf16;
+        a.qweight = qweight;
+        a.scales = static_cast<const uint16_t*>(scales_fp16);
+        a.zeros = nullptr;
+        a.Y = Y;
+        a.status = st.status;
+        a.M = (int)M;
+        a.N = (int)d_out;
+        a.K = (int)d_in;
+        a.g = group_size;
+        a.G = (int)(d_in / group_size);
+        a.symmetric = 1;
+        a.y_fp32 = y_dtype == WQ_OUT_FP32;
+        a.bits = 8;
+        LaunchOptions opt;
+        opt.pdl = false;
+        e = launch_gemm(a, st.num_sms, opt, s);
+    }
     return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
 

@@ -71,6 +71,7 @@ struct GemmArgs {
     int M, N, K, G, g;
     int symmetric;
     int y_fp32;
+    int bits;  // 4 (qweight [N][K/8], nibbles) or 8 (qweight [N][K/4], symmetric bytes)
 };
 
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, const LaunchOptions& opt, cudaStream_t stream);
@@ -87,6 +88,22 @@ cudaError_t launch_awq_loss(const float* Yref, const float* Y, int64_t n, double
                             cudaStream_t stream);
 cudaError_t launch_awq_select(const double* losses, int n, int32_t* best, cudaStream_t stream);
 int awq_loss_partials();
+
+// W8A16 (w8.cu): symmetric INT8 [-127, 127], 4 codes per word.
+struct W8Args {
+    const void* X;           // bf16 [M][K]
+    const uint32_t* qweight; // [N][K/4]
+    const uint16_t* scales;  // fp16 [N][G]
+    void* Y;                 // [M][N] bf16 or fp32
+    uint32_t* status;
+    int64_t N, K, G;
+    int M, g, y_fp32;
+};
+cudaError_t launch_quantize_w8(const void* W, int64_t N, int64_t K, int g, uint32_t* qweight, uint16_t* scales,
+                               uint32_t* status, int num_sms, cudaStream_t stream);
+cudaError_t launch_dequantize_w8(const uint32_t* qweight, const uint16_t* scales, int64_t N, int64_t K, int g,
+                                 void* out, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemv_w8a16(const W8Args& a, cudaStream_t stream);  // M <= 16
 
 // GPTQ (gptq.cu): scales/zeros must already hold the RTN parameters of W.
 size_t gptq_workspace_bytes(int64_t N, int64_t K);
