@@ -334,11 +334,12 @@ def run_ours(args, dist: Dist):
     T_CAL = 512
     Xc = syn.activations(T_CAL, D, 21, 2, "cuda", channel_outlier_frac=0.001)
     ws = torch.empty(b.wq_awq_workspace_bytes(D, D, T_CAL, G128), dtype=torch.uint8, device="cuda")
-    for _ in range(3):
+    short = args.steps < 20  # the short form (profiling runs) times each search once
+    for _ in range(1 if short else 3):
         r_awq = b.awq_search(W, Xc, workspace=ws)
     torch.cuda.synchronize()
     dist.barrier()
-    asteps = 5
+    asteps = 1 if short else 5
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
     for _ in range(asteps):
@@ -356,11 +357,11 @@ def run_ours(args, dist: Dist):
     # GPTQ (fp64 Hessian, inverse factor and error-feedback sweep), the page's
     # setting: symmetric, group 128, act-order; same calibration activations
     gws = torch.empty(b.wq_gptq_workspace_bytes(D, D), dtype=torch.uint8, device="cuda")
-    for _ in range(2):
+    for _ in range(1 if short else 2):
         p_g, _ = b.gptq(W, Xc, G128, True, True, workspace=gws)
     torch.cuda.synchronize()
     dist.barrier()
-    gsteps = 3
+    gsteps = 1 if short else 3
     ev0.record()
     for _ in range(gsteps):
         p_g, _ = b.gptq(W, Xc, G128, True, True, workspace=gws)
