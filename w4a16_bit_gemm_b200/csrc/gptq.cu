@@ -98,14 +98,30 @@ __global__ void __launch_bounds__(kTileThreads) gptq_hessian_kernel(const uint16
 }
 
 // Dampening: d = 0.01 mean(diag H) (diagonal summed in index order; d = 1 if
-// the mean is 0), added to every diagonal entry.  One thread.
-__global__ void gptq_damp_kernel(double* __restrict__ H, int64_t K) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    double s = 0.0;
-    for (int64_t j = 0; j < K; ++j) s = __dadd_rn(s, H[j * K + j]);
-    double d = __dmul_rn(0.01, __ddiv_rn(s, (double)K));
+// the mean is 0), added to every diagonal entry.  One CTA: the diagonal is
+// gathered into shared memory in parallel, then one thread sums it in order.
+constexpr int kDampThreads = 1024;
+constexpr int kDampChunk = 4096;
+
+__global__ void __launch_bounds__(kDampThreads) gptq_damp_kernel(double* __restrict__ H, int64_t K) {
+    __shared__ double diag[kDampChunk];
+    __shared__ double total;
+    if (threadIdx.x == 0) total = 0.0;
+    for (int64_t j0 = 0; j0 < K; j0 += kDampChunk) {
+        const int n = (int)(K - j0 < kDampChunk ? K - j0 : kDampChunk);
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += kDampThreads) diag[i] = H[(j0 + i) * K + j0 + i];
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double s = total;
+            for (int i = 0; i < n; ++i) s = __dadd_rn(s, diag[i]);
+            total = s;
+        }
+    }
+    __syncthreads();
+    double d = __dmul_rn(0.01, __ddiv_rn(total, (double)K));
     if (d == 0.0) d = 1.0;
-    for (int64_t j = 0; j < K; ++j) H[j * K + j] = __dadd_rn(H[j * K + j], d);
+    for (int64_t j = threadIdx.x; j < K; j += kDampThreads) H[j * K + j] = __dadd_rn(H[j * K + j], d);
 }
 
 // Processing order: by decreasing diagonal, ties in index order (the rank of
@@ -578,7 +594,7 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t N, int64_t K, const uint16_t*
     // H, dampening, processing order, permuted copy
     const unsigned tk = tiles(K);
     gptq_hessian_kernel<<<dim3(tk, tk), kTileThreads, 0, s>>>(X, T, K, B1);
-    gptq_damp_kernel<<<1, 32, 0, s>>>(B1, K);
+    gptq_damp_kernel<<<1, kDampThreads, 0, s>>>(B1, K);
     const unsigned kb = (unsigned)((K + 255) / 256);
     gptq_diag_check_kernel<<<kb, 256, 0, s>>>(B1, K, nonfinite);
     gptq_perm_kernel<<<kb, 256, 0, s>>>(B1, K, act_order, perm, nonfinite);
