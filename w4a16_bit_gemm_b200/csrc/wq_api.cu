@@ -122,6 +122,18 @@ CUresult encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const
                     swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+wq_status awq_check_args(const void* W_bf16, int64_t d_out, int64_t d_in, const void* X_bf16, int64_t T,
+                         int32_t group_size, int32_t symmetric, const uint32_t* qweight, const void* scales_fp16,
+                         const void* zeros_fp16, const void* s_bf16, const double* losses, const int32_t* best) {
+    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
+    if (v != WQ_OK) return v;
+    if (!W_bf16 || !X_bf16 || !s_bf16 || !aligned(W_bf16, 16) || !aligned(X_bf16, 16) || !aligned(s_bf16, 2))
+        return WQ_ERR_INVALID_ARG;
+    if (T < 1 || T > (1ll << 31) - 1 || (d_in % 8) != 0) return WQ_ERR_INVALID_ARG;
+    if ((losses && !aligned(losses, 8)) || (best && !aligned(best, 4))) return WQ_ERR_INVALID_ARG;
+    return WQ_OK;
+}
+
 }  // namespace wq
 
 using namespace wq;
@@ -301,13 +313,10 @@ wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const v
                         int32_t group_size, int32_t symmetric, uint32_t* qweight, void* scales_fp16,
                         void* zeros_fp16, void* s_bf16, double* losses, int32_t* best, void* workspace,
                         size_t workspace_bytes, void* stream) {
-    wq_status v = check_artifact(qweight, scales_fp16, zeros_fp16, d_out, d_in, group_size, symmetric);
+    wq_status v = awq_check_args(W_bf16, d_out, d_in, X_bf16, T, group_size, symmetric, qweight, scales_fp16,
+                                 zeros_fp16, s_bf16, losses, best);
     if (v != WQ_OK) return v;
-    if (!W_bf16 || !X_bf16 || !s_bf16 || !workspace || !aligned(W_bf16, 16) || !aligned(X_bf16, 16) ||
-        !aligned(s_bf16, 2) || !aligned(workspace, 256))
-        return WQ_ERR_INVALID_ARG;
-    if (T < 1 || T > (1ll << 31) - 1 || (d_in % 8) != 0) return WQ_ERR_INVALID_ARG;
-    if ((losses && !aligned(losses, 8)) || (best && !aligned(best, 4))) return WQ_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256)) return WQ_ERR_INVALID_ARG;
     const AwqWorkspace L = awq_workspace(d_out, d_in, T, group_size);
     if (workspace_bytes < L.total) return WQ_ERR_INVALID_ARG;
     DeviceState st;

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/wq.h"
+
 namespace wq {
 
 cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric, uint32_t* qweight,
@@ -88,6 +90,10 @@ cudaError_t launch_awq_loss(const float* Yref, const float* Y, int64_t n, double
                             cudaStream_t stream);
 cudaError_t launch_awq_select(const double* losses, int n, int32_t* best, cudaStream_t stream);
 int awq_loss_partials();
+// Argument checks of the AWQ search (everything except the workspace).
+wq_status awq_check_args(const void* W_bf16, int64_t d_out, int64_t d_in, const void* X_bf16, int64_t T,
+                         int32_t group_size, int32_t symmetric, const uint32_t* qweight, const void* scales_fp16,
+                         const void* zeros_fp16, const void* s_bf16, const double* losses, const int32_t* best);
 
 // W8A16 (w8.cu): symmetric INT8 [-127, 127], 4 codes per word.
 struct W8Args {
