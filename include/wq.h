@@ -238,6 +238,23 @@ wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const v
 size_t wq_awq_workspace_bytes(int64_t d_out, int64_t d_in, int64_t T, int32_t group_size);
 
 /*
+ * wq_awq_search_static -- wq_awq_search without a caller workspace: the
+ * scratch is a device array owned by the library (wq_awq_static_scratch_bytes()
+ * bytes, reserved on a device when a process first calls this function).
+ * Arguments, results and errors as wq_awq_search, plus WQ_ERR_UNSUPPORTED
+ * when wq_awq_workspace_bytes(d_out, d_in, T, group_size) exceeds the array.
+ * All calls on a device share the array: they must not overlap in time
+ * (queue them on one stream).
+ */
+wq_status wq_awq_search_static(const void* W_bf16, int64_t d_out, int64_t d_in, const void* X_bf16,
+                               int64_t T, int32_t group_size, int32_t symmetric, uint32_t* qweight,
+                               void* scales_fp16, void* zeros_fp16, void* s_bf16, double* losses,
+                               int32_t* best, void* stream);
+
+/* Size of the library-owned scratch of wq_awq_search_static, in bytes. */
+size_t wq_awq_static_scratch_bytes(void);
+
+/*
  * wq_awq_scale_activations -- X'[t][j] = bf16_rn(fl32(X[t][j] / s_j)), the
  * activation side of the AWQ scaling identity.  X_bf16 and Xp_bf16 are
  * [T][d_in] bf16, 16-byte aligned (they may not overlap unless equal);

@@ -168,3 +168,11 @@ def test_w8_linear_and_dequant_reject(lib):
     assert lib.wq_linear_w8a16(FAKE, 1, FAKE, FAKE, 64, 256, 256, FAKE, 3, None) == 1
     assert lib.wq_dequantize_w8(FAKE, FAKE, 4, 256, 128, None, None) == 1
     assert lib.wq_dequantize_w8(FAKE, None, 4, 256, 128, FAKE, None) == 1
+
+
+def test_awq_static_rejects_before_any_device_work(lib):
+    # a layer whose scratch exceeds the library-owned array
+    assert lib.wq_awq_static_scratch_bytes() >= 64 << 20
+    st = lib.wq_awq_search_static(FAKE, 8192, 8192, FAKE, 512, 128, 0, FAKE, FAKE, FAKE, FAKE, None, None, None)
+    assert st == 2
+    assert lib.wq_awq_search_static(None, 64, 256, FAKE, 8, 128, 0, FAKE, FAKE, FAKE, FAKE, None, None, None) == 1

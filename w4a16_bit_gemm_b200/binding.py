@@ -62,6 +62,10 @@ def _load() -> ctypes.CDLL:
     lib.wq_awq_search.restype = ctypes.c_int
     lib.wq_awq_workspace_bytes.argtypes = [i64, i64, i64, i32]
     lib.wq_awq_workspace_bytes.restype = sz
+    lib.wq_awq_search_static.argtypes = [P, i64, i64, P, i64, i32, i32, P, P, P, P, P, P, P]
+    lib.wq_awq_search_static.restype = ctypes.c_int
+    lib.wq_awq_static_scratch_bytes.argtypes = []
+    lib.wq_awq_static_scratch_bytes.restype = sz
     lib.wq_awq_scale_activations.argtypes = [P, i64, i64, P, P, P]
     lib.wq_awq_scale_activations.restype = ctypes.c_int
     lib.wq_quantize_w8.argtypes = [P, i64, i64, i32, P, P, P]
@@ -141,6 +145,12 @@ def wq_awq_search(W, d_out, d_in, X, T, group_size, symmetric, qweight, scales, 
     return lib.wq_awq_search(_ptr(W), d_out, d_in, _ptr(X), T, group_size, int(symmetric), _ptr(qweight),
                              _ptr(scales), _ptr(zeros), _ptr(s), _ptr(losses), _ptr(best), _ptr(workspace),
                              workspace_bytes, _stream(stream))
+
+
+def wq_awq_search_static(W, d_out, d_in, X, T, group_size, symmetric, qweight, scales, zeros, s, losses, best,
+                         stream=None) -> int:
+    return lib.wq_awq_search_static(_ptr(W), d_out, d_in, _ptr(X), T, group_size, int(symmetric), _ptr(qweight),
+                                    _ptr(scales), _ptr(zeros), _ptr(s), _ptr(losses), _ptr(best), _stream(stream))
 
 
 def wq_awq_workspace_bytes(d_out, d_in, T, group_size) -> int:
@@ -365,6 +375,26 @@ def gptq(W: torch.Tensor, X: torch.Tensor, group_size: int = 128, symmetric: boo
     _check(wq_gptq(W, d_out, d_in, X, X.shape[0], group_size, symmetric, act_order, out.qweight, out.scales,
                    out.zeros, perm, workspace, workspace.numel() * workspace.element_size(), stream), "wq_gptq")
     return out, perm
+
+
+def awq_search_static(W: torch.Tensor, X: torch.Tensor, group_size: int = 128, symmetric: bool = False,
+                      stream=None) -> AWQResult:
+    """awq_search with the library-owned scratch instead of a workspace tensor."""
+    _require_cuda(W, X)
+    if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D bf16 CUDA tensor")
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or not X.is_contiguous() or X.shape[1] != W.shape[1]:
+        raise ValueError("X must be a contiguous [T, d_in] bf16 CUDA tensor")
+    d_out, d_in = W.shape
+    if d_in % group_size != 0:
+        raise ValueError("group_size must divide d_in")
+    out = alloc_packed(d_out, d_in, group_size, symmetric, W.device)
+    s = torch.empty(d_in, dtype=torch.bfloat16, device=W.device)
+    losses = torch.empty(11, dtype=torch.float64, device=W.device)
+    best = torch.empty(1, dtype=torch.int32, device=W.device)
+    _check(wq_awq_search_static(W, d_out, d_in, X, X.shape[0], group_size, symmetric, out.qweight, out.scales,
+                                out.zeros, s, losses, best, stream), "wq_awq_search_static")
+    return AWQResult(out, s, losses, best)
 
 
 def awq_scale_activations(X: torch.Tensor, s: torch.Tensor, out: torch.Tensor | None = None,
