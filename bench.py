@@ -93,17 +93,25 @@ def load_peaks():
 # --------------------------------------------------------------------------
 
 class Dist:
+    """One process per GPU (RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* from the
+    launcher).  The backend is NCCL; WQ_DIST_BACKEND=gloo runs the same
+    plumbing on CPU processes (tests)."""
+
     def __init__(self):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = os.environ.get("WQ_DIST_BACKEND", "nccl")
         self.pg = False
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            if self.backend == "nccl":
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                        device_id=torch.device("cuda", self.local))
+            else:
+                dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120))
             self.pg = True
 
     def barrier(self):
@@ -115,7 +123,7 @@ class Dist:
         if not self.pg:
             return v
         import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device="cuda" if self.backend == "nccl" else "cpu")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
