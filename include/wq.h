@@ -73,7 +73,7 @@ extern "C" {
 typedef enum {
     WQ_OK = 0,
     WQ_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or group size */
-    WQ_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+    WQ_ERR_UNSUPPORTED = 2, /* valid request the library does not implement */
     WQ_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
     WQ_ERR_NONFINITE = 4,   /* returned by wq_get_device_error: NaN/Inf input seen */
     WQ_ERR_TIMEOUT = 5,     /* returned by wq_get_device_error: a device wait gave up */
