@@ -39,7 +39,7 @@ constexpr int kTile = 64;        // output tile edge of the fp64 tiled kernels
 constexpr int kTileThreads = 256;  // 16 x 16 threads, 4 x 4 entries each
 constexpr int kPanel = 32;       // Cholesky panel width / inverse row block
 constexpr int kChunk = 32;       // inner-dimension chunk staged in shared memory
-constexpr int kSweepWarps = 16;  // rows per sweep CTA (one warp per row)
+constexpr int kSweepWarps = 32;  // rows per sweep CTA (one warp per row)
 
 __device__ __forceinline__ double bf16_bits_to_f64(uint16_t b) {
     return (double)__uint_as_float((uint32_t)b << 16);
@@ -163,18 +163,23 @@ __global__ void gptq_gather_kernel(const double* __restrict__ H, const int32_t* 
 // ---------------------------------------------------------------------------
 
 // The panel's diagonal block: one CTA of kPanel threads, column by column.
-__global__ void __launch_bounds__(kPanel) gptq_chol_diag_kernel(double* __restrict__ A, int64_t K, int64_t p0,
-                                                                uint32_t* __restrict__ status) {
+constexpr int kDiagThreads = 256;
+
+__global__ void __launch_bounds__(kDiagThreads) gptq_chol_diag_kernel(double* __restrict__ A, int64_t K, int64_t p0,
+                                                                      uint32_t* __restrict__ status) {
+    // right-looking inside the block: after column j is final, every later
+    // entry (i, c) of the block takes its term l[i][j] l[c][j] in turn, so
+    // each entry still receives its terms in ascending j
     __shared__ double Ls[kPanel][kPanel + 1];
     const int w = (int)(K - p0 < kPanel ? K - p0 : kPanel);
-    const int i = threadIdx.x;
-    if (i < w)
-        for (int c = 0; c <= i; ++c) Ls[i][c] = A[(p0 + i) * K + p0 + c];
+    for (int e = threadIdx.x; e < kPanel * kPanel; e += kDiagThreads) {
+        const int r = e / kPanel, c = e % kPanel;
+        if (r < w && c <= r) Ls[r][c] = A[(p0 + r) * K + p0 + c];
+    }
     __syncthreads();
     for (int j = 0; j < w; ++j) {
-        if (i == j) {
+        if (threadIdx.x == 0) {
             double d = Ls[j][j];
-            for (int k = 0; k < j; ++k) d = __dsub_rn(d, __dmul_rn(Ls[j][k], Ls[j][k]));
             if (!(d > 0.0) || !isfinite(d)) {
                 d = 1.0;
                 raise_flag(status, WQ_DEVFLAG_RANGE);
@@ -182,15 +187,20 @@ __global__ void __launch_bounds__(kPanel) gptq_chol_diag_kernel(double* __restri
             Ls[j][j] = __dsqrt_rn(d);
         }
         __syncthreads();
-        if (i > j && i < w) {
-            double v = Ls[i][j];
-            for (int k = 0; k < j; ++k) v = __dsub_rn(v, __dmul_rn(Ls[i][k], Ls[j][k]));
-            Ls[i][j] = __ddiv_rn(v, Ls[j][j]);
+        for (int i = j + 1 + (int)threadIdx.x; i < w; i += kDiagThreads) Ls[i][j] = __ddiv_rn(Ls[i][j], Ls[j][j]);
+        __syncthreads();
+        // trailing entries (i, c), j < c <= i < w
+        const int m = w - j - 1;
+        for (int e = threadIdx.x; e < m * m; e += kDiagThreads) {
+            const int i = j + 1 + e / m, c = j + 1 + e % m;
+            if (c <= i) Ls[i][c] = __dsub_rn(Ls[i][c], __dmul_rn(Ls[i][j], Ls[c][j]));
         }
         __syncthreads();
     }
-    if (i < w)
-        for (int c = 0; c <= i; ++c) A[(p0 + i) * K + p0 + c] = Ls[i][c];
+    for (int e = threadIdx.x; e < kPanel * kPanel; e += kDiagThreads) {
+        const int r = e / kPanel, c = e % kPanel;
+        if (r < w && c <= r) A[(p0 + r) * K + p0 + c] = Ls[r][c];
+    }
 }
 
 // Rows below the diagonal block: one thread per row.
@@ -204,17 +214,22 @@ __global__ void __launch_bounds__(128) gptq_chol_panel_kernel(double* __restrict
     __syncthreads();
     const int64_t i = p0 + w + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= K) return;
+    // the row's panel entries in registers; right-looking: once entry j is
+    // final, the later entries take their term row[j] l[c][j] in turn
     double row[kPanel];
+#pragma unroll
+    for (int j = 0; j < kPanel; ++j) row[j] = j < w ? A[i * K + p0 + j] : 0.0;
 #pragma unroll
     for (int j = 0; j < kPanel; ++j) {
         if (j < w) {
-            double v = A[i * K + p0 + j];
+            row[j] = __ddiv_rn(row[j], Ls[j][j]);
 #pragma unroll
-            for (int k = 0; k < j; ++k) v = __dsub_rn(v, __dmul_rn(row[k], Ls[j][k]));
-            row[j] = __ddiv_rn(v, Ls[j][j]);
-            A[i * K + p0 + j] = row[j];
+            for (int c = j + 1; c < kPanel; ++c) row[c] = __dsub_rn(row[c], __dmul_rn(row[j], Ls[c][j]));
         }
     }
+#pragma unroll
+    for (int j = 0; j < kPanel; ++j)
+        if (j < w) A[i * K + p0 + j] = row[j];
 }
 
 // Trailing update: A[i][c] -= l[i][k] l[c][k], k = p0 .. p1-1 in turn, for
@@ -280,23 +295,23 @@ __global__ void __launch_bounds__(128) gptq_trinv_block_kernel(const double* __r
     __syncthreads();
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (j >= r0 + w) return;
-    double col[kPanel];  // Linv[r0 + k][j] of this block
+    // acc[ii]: the accumulator of entry (r0 + ii, j); right-looking: once
+    // Linv[r0 + ii][j] is final, the later rows of the block take their term
+    // l[r0 + i2][r0 + ii] Linv[r0 + ii][j] in turn (terms with r0 + ii < j are
+    // skipped: the sum of entry (i, j) starts at k = j)
+    double acc[kPanel];
+#pragma unroll
+    for (int ii = 0; ii < kPanel; ++ii) acc[ii] = (ii < w && r0 + ii > j) ? Li[(r0 + ii) * K + j] : 0.0;
 #pragma unroll
     for (int ii = 0; ii < kPanel; ++ii) {
         if (ii < w) {
             const int64_t i = r0 + ii;
-            double out = 0.0;
-            if (i == j) {
-                out = __ddiv_rn(1.0, Ls[ii][ii]);
-            } else if (i > j) {
-                double v = Li[i * K + j];
+            if (i >= j) {
+                const double out = i == j ? __ddiv_rn(1.0, Ls[ii][ii]) : __ddiv_rn(-acc[ii], Ls[ii][ii]);
+                Li[i * K + j] = out;
 #pragma unroll
-                for (int k = 0; k < ii; ++k)
-                    if (r0 + k >= j) v = __dadd_rn(v, __dmul_rn(Ls[ii][k], col[k]));
-                out = __ddiv_rn(-v, Ls[ii][ii]);
+                for (int i2 = ii + 1; i2 < kPanel; ++i2) acc[i2] = __dadd_rn(acc[i2], __dmul_rn(Ls[i2][ii], out));
             }
-            col[ii] = out;
-            if (i >= j) Li[i * K + j] = out;
         }
     }
 }
@@ -552,7 +567,7 @@ unsigned tiles(int64_t n) { return (unsigned)((n + kTile - 1) / kTile); }
 
 cudaError_t cholesky_lower(double* A, int64_t K, uint32_t* status, cudaStream_t s) {
     for (int64_t p0 = 0; p0 < K; p0 += kPanel) {
-        gptq_chol_diag_kernel<<<1, kPanel, 0, s>>>(A, K, p0, status);
+        gptq_chol_diag_kernel<<<1, kDiagThreads, 0, s>>>(A, K, p0, status);
         const int64_t p1 = p0 + kPanel;
         if (p1 >= K) break;
         gptq_chol_panel_kernel<<<(unsigned)((K - p1 + 127) / 128), 128, 0, s>>>(A, K, p0);
