@@ -383,22 +383,25 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_large_group_kernel(
 // into 64 bytes of bf16, using the exact bf16x2 dequantization shared with the
 // linear-layer kernels.  Grid-stride with two quads in flight per thread.
 constexpr int kDeqThreads = 256;
-constexpr int kDeqPerThread = 2;
+constexpr int kDeqPerThread = 2;  // 2-word units in flight per thread
 
+// One thread per unit of 2 packed words (16 weights, always inside one group
+// because g is a multiple of 32): an 8-byte load and two 16-byte stores, so a
+// warp reads 256 contiguous bytes and writes 1 KB contiguous.
 __global__ void __launch_bounds__(kDeqThreads) dequantize_kernel(
-    const uint4* __restrict__ qweight, const uint16_t* __restrict__ scales,
-    const uint16_t* __restrict__ zeros, int64_t nquad, int g, int symmetric, uint4* __restrict__ W_hat) {
+    const uint2* __restrict__ qweight, const uint16_t* __restrict__ scales,
+    const uint16_t* __restrict__ zeros, int64_t npair, int g, int symmetric, uint4* __restrict__ W_hat) {
     const int64_t stride = (int64_t)gridDim.x * (kDeqThreads * kDeqPerThread);
-    for (int64_t base = (int64_t)blockIdx.x * (kDeqThreads * kDeqPerThread) + threadIdx.x; base < nquad;
+    for (int64_t base = (int64_t)blockIdx.x * (kDeqThreads * kDeqPerThread) + threadIdx.x; base < npair;
          base += stride) {
-        uint4 q[kDeqPerThread];
+        uint2 q[kDeqPerThread];
         uint16_t s16[kDeqPerThread], z16[kDeqPerThread];
 #pragma unroll
         for (int u = 0; u < kDeqPerThread; ++u) {
             const int64_t t = base + (int64_t)u * kDeqThreads;
-            if (t < nquad) {
-                q[u] = ld_nc_v4(qweight + t);
-                const int64_t gi = (t * 32) / g;
+            if (t < npair) {
+                q[u] = __ldg(qweight + t);
+                const int64_t gi = (t * 16) / g;
                 s16[u] = scales[gi];
                 z16[u] = symmetric ? (uint16_t)0 : zeros[gi];
             }
@@ -406,16 +409,14 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_kernel(
 #pragma unroll
         for (int u = 0; u < kDeqPerThread; ++u) {
             const int64_t t = base + (int64_t)u * kDeqThreads;
-            if (t >= nquad) continue;
+            if (t >= npair) continue;
             const int z = symmetric ? 0 : (int)__half2float(__ushort_as_half(z16[u]));
             const GroupConsts c = make_group_consts(s16[u], z, symmetric != 0);
-            const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint32_t o[4];
-                dequant_word_natural(w[j], c, o);
-                W_hat[t * 4 + j] = make_uint4(o[0], o[1], o[2], o[3]);
-            }
+            uint32_t o[4], o2[4];
+            dequant_word_natural(q[u].x, c, o);
+            dequant_word_natural(q[u].y, c, o2);
+            W_hat[t * 2] = make_uint4(o[0], o[1], o[2], o[3]);
+            W_hat[t * 2 + 1] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
         }
     }
 }
@@ -597,11 +598,11 @@ cudaError_t launch_quantize_clip(const void* W, int64_t d_out, int64_t d_in, int
 cudaError_t launch_dequantize(const uint32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
                               int64_t d_out, int64_t d_in, int g, int symmetric, void* W_hat, int num_sms,
                               cudaStream_t stream) {
-    const int64_t nquad = d_out * d_in / 32;
-    int64_t blocks = (nquad + kDeqThreads * kDeqPerThread - 1) / (kDeqThreads * kDeqPerThread);
+    const int64_t npair = d_out * d_in / 16;
+    int64_t blocks = (npair + kDeqThreads * kDeqPerThread - 1) / (kDeqThreads * kDeqPerThread);
     if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
-    dequantize_kernel<<<blocks, kDeqThreads, 0, stream>>>(reinterpret_cast<const uint4*>(qweight), scales, zeros,
-                                                          nquad, g, symmetric, static_cast<uint4*>(W_hat));
+    dequantize_kernel<<<blocks, kDeqThreads, 0, stream>>>(reinterpret_cast<const uint2*>(qweight), scales, zeros,
+                                                          npair, g, symmetric, static_cast<uint4*>(W_hat));
     return cudaGetLastError();
 }
 

@@ -15,7 +15,7 @@
 //       complement, low byte first; scales fp16 [d_out][d_in / g].
 //
 // The linear layer for M <= 16 is a split-K GEMV on mma.sync m16n8k16: a CTA
-// owns 16 output rows, its 8 warps split d_in, lane (r, t) dequantizes 16
+// owns 16 output rows, its 16 warps split d_in, lane (r, t) dequantizes 16
 // consecutive codes of rows r and r + 8 straight into bf16x2 A fragments and
 // reads the matching activation pairs as B fragments (the sum over k is order
 // free, so each lane group t may own its own column chunks); partial sums
@@ -127,10 +127,10 @@ __global__ void __launch_bounds__(256) dequantize_w8_kernel(const uint32_t* __re
 // ---------------------------------------------------------------------------
 // GEMV, M <= 16 (NT = 1: M <= 8, NT = 2: M <= 16).
 // ---------------------------------------------------------------------------
-constexpr int kGemvWarps = 8;
+constexpr int kGemvWarps = 16;
 
 template <int NT>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv_w8a16_kernel(const W8Args a) {
+__global__ void __launch_bounds__(kGemvWarps * 32, 2) gemv_w8a16_kernel(const W8Args a) {
     __shared__ float red[kGemvWarps][16][16];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, t = lane & 3;
@@ -148,32 +148,44 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_w8a16_kernel(const W8Arg
     float d[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0.0f;
-#pragma unroll 2
-    for (int64_t i = 0; i < iters; ++i) {
-        const int64_t c = c_begin + t + 4 * i;
-        const bool live = c < c_end;
-        const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-        const uint4 wa = (live && vA) ? ld_nc_v4(qA + c) : zero;
-        const uint4 wb = (live && vB) ? ld_nc_v4(qB + c) : zero;
-        const int64_t gi = live ? (c * 16) / a.g : 0;
-        const float s_a = (live && vA) ? __half2float(__ushort_as_half(sA[gi])) : 0.0f;
-        const float s_b = (live && vB) ? __half2float(__ushort_as_half(sB[gi])) : 0.0f;
-        uint32_t fa[8], fb[8];
-        dequant16_w8(wa, s_a, fa);
-        dequant16_w8(wb, s_b, fb);
+    // the weight loads of kPre chunks are issued before any is used
+    constexpr int kPre = NT == 1 ? 2 : 1;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t i0 = 0; i0 < iters; i0 += kPre) {
+        uint4 wa[kPre], wb[kPre];
+        float s_a[kPre], s_b[kPre];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int m = r + 8 * nt;
-            uint4 x0 = zero, x1 = zero;
-            if (live && m < a.M) {
-                const uint4* xp = reinterpret_cast<const uint4*>(X + (int64_t)m * a.K + c * 16);
-                x0 = __ldg(xp);
-                x1 = __ldg(xp + 1);
+        for (int u = 0; u < kPre; ++u) {
+            const int64_t c = c_begin + t + 4 * (i0 + u);
+            const bool live = (i0 + u) < iters && c < c_end;
+            wa[u] = (live && vA) ? ld_nc_v4(qA + c) : zero;
+            wb[u] = (live && vB) ? ld_nc_v4(qB + c) : zero;
+            const int64_t gi = live ? (c * 16) / a.g : 0;
+            s_a[u] = (live && vA) ? __half2float(__ushort_as_half(sA[gi])) : 0.0f;
+            s_b[u] = (live && vB) ? __half2float(__ushort_as_half(sB[gi])) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kPre; ++u) {
+            const int64_t c = c_begin + t + 4 * (i0 + u);
+            const bool live = (i0 + u) < iters && c < c_end;
+            uint32_t fa[8], fb[8];
+            dequant16_w8(wa[u], s_a[u], fa);
+            dequant16_w8(wb[u], s_b[u], fb);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int m = r + 8 * nt;
+                uint4 x0 = zero, x1 = zero;
+                if (live && m < a.M) {
+                    const uint4* xp = reinterpret_cast<const uint4*>(X + (int64_t)m * a.K + c * 16);
+                    x0 = __ldg(xp);
+                    x1 = __ldg(xp + 1);
+                }
+                const uint32_t xb[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mma_bf16_16816(d[nt], fa[2 * j], fb[2 * j], fa[2 * j + 1], fb[2 * j + 1], xb[2 * j],
+                                   xb[2 * j + 1]);
             }
-            const uint32_t xb[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_bf16_16816(d[nt], fa[2 * j], fb[2 * j], fa[2 * j + 1], fb[2 * j + 1], xb[2 * j], xb[2 * j + 1]);
         }
     }
     // d[nt]: (row r, token 8nt + 2t), (r, 8nt + 2t + 1), (r + 8, 8nt + 2t), (r + 8, 8nt + 2t + 1)
@@ -185,9 +197,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_w8a16_kernel(const W8Arg
         red[warp][r + 8][8 * nt + 2 * t + 1] = d[nt][3];
     }
     __syncthreads();
+    // 16 rows x 16 tokens: the first 256 threads finish one output each
     const int rr = threadIdx.x >> 4, m = threadIdx.x & 15;
     const int64_t n = n0 + rr;
-    if (m < a.M && m < 8 * NT && n < a.N) {
+    if (threadIdx.x < 256 && m < a.M && m < 8 * NT && n < a.N) {
         float y = 0.0f;
 #pragma unroll
         for (int w = 0; w < kGemvWarps; ++w) y += red[w][rr][m];
