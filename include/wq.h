@@ -1,6 +1,8 @@
 /*
- * wq.h -- C ABI of libwq: group-wise RTN 4-bit weight quantization,
- * dequantization and W4A16 linear layers on NVIDIA B200 (sm_100a).
+ * wq.h -- C ABI of libwq: group-wise 4-bit weight quantization (RTN, with an
+ * MSE-optimal clipping search, AWQ scaling or GPTQ error feedback),
+ * dequantization and W4A16 linear layers, plus the INT8 (W8A16) variant, on
+ * NVIDIA B200 (sm_100a).
  *
  * The operations are the ones defined on
  *   "LLM Quantization: GPTQ, AWQ, SmoothQuant, FP8, KV Cache (7/10)"
@@ -16,10 +18,13 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - All array arguments are DEVICE pointers owned by the caller.  The library
- *   never frees or retains them.  The library owns only one device status
- *   word per device (a static device variable; no entry point allocates
- *   device memory).  The first call on a device looks up that word's address
- *   and should not be made inside a stream capture.
+ *   never frees or retains them.  The library owns one device status word per
+ *   device (a static device variable) and, only once wq_awq_search_static is
+ *   called, that function's static scratch array; wq_awq_search's reference
+ *   GEMM runs in cuBLAS, which allocates its own workspace on first use.  No
+ *   other entry point allocates device memory.  The first call on a device
+ *   looks up the status word's address and should not be made inside a
+ *   stream capture.
  * - Matrices are dense row-major.  bf16 and fp16 values are passed as their
  *   16-bit storage (void*).
  * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
