@@ -919,7 +919,12 @@ int wqo_pack8(const int32_t* codes, int64_t d_out, int64_t d_in, uint32_t* qweig
     for (int64_t r = 0; r < d_out; ++r)
         for (int64_t c4 = 0; c4 < d_in / 4; ++c4) {
             uint32_t w = 0;
-            for (int j = 0; j < 4; ++j) w |= ((uint32_t)codes[r * d_in + c4 * 4 + j] & 0xffu) << (8 * j);
+            for (int j = 0; j < 4; ++j)
+#if WQO_MUTANT == 8 /* mistake: high byte first */
+                w |= ((uint32_t)codes[r * d_in + c4 * 4 + j] & 0xffu) << (8 * (3 - j));
+#else
+                w |= ((uint32_t)codes[r * d_in + c4 * 4 + j] & 0xffu) << (8 * j);
+#endif
             qweight[r * (d_in / 4) + c4] = w;
         }
     return 0;

@@ -1,7 +1,7 @@
 """Planted mistakes: each mutant of the oracle (one plausible error compiled
 in with -DWQO_MUTANT=k) must fail at least one pin, and the real oracle must
 pass the same pins.  This shows the pins constrain every step: statistics,
-scale, zero point, rounding, packing, dequantization, the linear layer and
+scale, zero point, rounding, 4- and 8-bit packing, dequantization, the linear layer and
 the clipping search (error formula and selection), the AWQ scales and
 GPTQ (pivot division, tail update, processing order)."""
 import pytest
@@ -20,6 +20,7 @@ PINS = [
     lambda: pins.test_brute_force_argmin(-1.0, 1.5, False),
     lambda: pins.test_brute_force_argmin(0.25, 7.0, False),
     pins.test_pack_layout_low_nibble_first,
+    pins.test_pack8_layout_low_byte_first,
     pins.test_dequant_exhaustive_against_library_rounding,
     pins.test_linear_special_cases_and_matmul,
     clip_pins.test_error_formula_is_the_exact_sum_of_squares,
@@ -40,6 +41,7 @@ MUTANTS = {
     5: "transposed weight in linear",
     6: "zero point dropped in dequant",
     7: "high nibble first",
+    8: "8-bit packing high byte first",
     9: "clip search sums absolute errors",
     10: "clip search keeps the largest error",
     11: "AWQ scales inverted",

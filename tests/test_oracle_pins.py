@@ -472,3 +472,26 @@ def test_whole_model_artifact_bytes():
     assert payload == 3_238_002_688 and sb + zb == 202_375_168
     assert payload + sb + zb == 3_440_377_856
     assert (payload + sb + zb) * 8 / P == 4.25
+
+
+# --------------------------------------------------------------------------
+# Monotonicity: within a group, a larger weight never gets a smaller code
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,symmetric,narrow", [(4, False, False), (4, True, False), (8, True, True)])
+def test_codes_are_monotone_within_a_group(bits, symmetric, narrow):
+    """[P1] Affine Quantization: q = clamp(round(x/s) + z) is non-decreasing in
+    x for s > 0, and so is x_hat = s (q - z)."""
+    rng = np.random.default_rng(11)
+    g = 128
+    x = rng.laplace(0, 0.02, (64, g)).astype(np.float32)
+    x[::7, 0] = 0.5  # a few outliers
+    W = bf16_bits(x)
+    codes, scales, zeros, _ = oracle.quantize(W, g, bits=bits, symmetric=symmetric, narrow=narrow)
+    vals = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).float().numpy()
+    W_hat = oracle.dequantize(codes, scales, zeros, g)
+    hat = torch.from_numpy(W_hat.view(np.int16)).view(torch.bfloat16).float().numpy()
+    for r in range(W.shape[0]):
+        order = np.argsort(vals[r], kind="stable")
+        assert np.all(np.diff(codes[r][order]) >= 0), r
+        assert np.all(np.diff(hat[r][order]) >= 0), r
