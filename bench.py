@@ -393,6 +393,47 @@ def run_ours(args, dist: Dist):
     td = dist.max(timed_graph(gd, qsteps, 3, dist)) / (qsteps * QC)
     secondary["dequantize"] = {"shape": "4096x4096", "GBps": qb / td / 1e9, "us_per_launch": td * 1e6,
                                "frac_of_measured_hbm": qb / td / 1e9 / hbm}
+    # references for the same M=1 layer: the pages' path B (full dequantize,
+    # then a bf16 matmul) and the unquantized bf16 layer, both through
+    # torch.matmul; timed locally (no collective), and an error in a reference
+    # leg is reported instead of stopping the benchmark
+    try:
+        Xr = syn.case_activations(syn.ATTN, 0, 1, "cuda")
+        Yr = [torch.empty(1, D, dtype=torch.bfloat16, device="cuda") for _ in range(QC)]
+
+        def path_b():
+            for i in range(QC):
+                b.dequantize(qpacks[i], out=What[i])
+                torch.matmul(Xr, What[i].t(), out=Yr[i])
+
+        def dense():
+            for i in range(QC):
+                torch.matmul(Xr, Ws[i].t(), out=Yr[i])
+
+        def local_time(graph, reps):
+            for _ in range(3):
+                graph.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / 1e3 / (reps * QC)
+
+        t_pb = local_time(capture(path_b), qsteps)
+        t_dn = local_time(capture(dense), qsteps)
+        secondary["references_m1"] = {
+            "shape": "4096x4096", "M": 1, "copies": QC,
+            "path_b_dequantize_then_matmul_us": t_pb * 1e6,
+            "bf16_matmul_us": t_dn * 1e6,
+            "bf16_matmul_GBps": (D * D * 2 + 2 * 2 * D) / t_dn / 1e9,
+            "w4a16_gemv_speedup_vs_bf16": t_dn / per_launch,
+            "w4a16_gemv_speedup_vs_path_b": t_pb / per_launch}
+        del Yr
+    except Exception as ex:  # noqa: BLE001
+        secondary["references_m1"] = {"error": repr(ex)[:300]}
     del gq, gd, Ws, qpacks, What, W
     torch.cuda.empty_cache()
 
@@ -501,9 +542,10 @@ def run_ours(args, dist: Dist):
 # CPU oracle (baseline and reference arm)
 # --------------------------------------------------------------------------
 
-def oracle_gemv_sample(n_launch: int):
+def oracle_gemv_sample(n_launch: int, nthreads: int | None = None):
     """The oracle as it stands on the same workload: for each launch of the
-    sample, unpack the artifact, dequantize and run the fp64 linear layer."""
+    sample, unpack the artifact, dequantize and run the fp64 linear layer
+    (on every host core unless nthreads is given)."""
     import oracle
     from w4a16_bit_gemm_b200 import synthetic as syn
     W = syn.case_weight(syn.ATTN, 0, "cpu")
@@ -511,7 +553,7 @@ def oracle_gemv_sample(n_launch: int):
     q, s, z, _, _ = oracle.quantize_pack4(Wb, 128, False)
     X = syn.activations(1, D, syn.ATTN.seed, 77, "cpu", channel_outlier_frac=0.001)
     Xb = X.view(torch.int16).numpy().view(np.uint16)
-    nthreads = oracle.default_threads()
+    nthreads = nthreads or oracle.default_threads()
     t0 = time.perf_counter()
     for _ in range(n_launch):
         codes = oracle.unpack4(q, D, False)
@@ -576,9 +618,12 @@ def main():
             out = run_ours(args, dist)
             if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
                 v, n, dt, nl = calibrated_sample()
+                v1, _, dt1 = oracle_gemv_sample(2, nthreads=1)
                 out["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": n, "kind": "oracle",
                                        "sample": f"{nl} GEMV launch(es) of the 4096x4096 M=1 workload "
-                                                 f"(unpack + dequantize + fp64 linear), {dt:.1f} s"}
+                                                 f"(unpack + dequantize + fp64 linear), {dt:.1f} s",
+                                       "single_thread_value": v1,
+                                       "single_thread_sample": f"2 launches on 1 core, {dt1:.1f} s"}
         if out is not None and dist.rank == 0:
             print(json.dumps(out), flush=True)
     finally:
