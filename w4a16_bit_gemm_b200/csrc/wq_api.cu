@@ -322,13 +322,6 @@ wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const v
     DeviceState st;
     if ((v = device_state(&st)) != WQ_OK) return v;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cublasHandle_t h;
-    {
-        std::lock_guard<std::mutex> lk(g_blas_mu);
-        if (!g_blas[st.dev] && cublasCreate(&g_blas[st.dev]) != CUBLAS_STATUS_SUCCESS) return WQ_ERR_CUDA;
-        h = g_blas[st.dev];
-        if (cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS) return WQ_ERR_CUDA;
-    }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint16_t* Wp = reinterpret_cast<uint16_t*>(ws + L.wp);
     uint32_t* qa = reinterpret_cast<uint32_t*>(ws + L.qa);
@@ -346,12 +339,20 @@ wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const v
     const uint16_t* W = static_cast<const uint16_t*>(W_bf16);
     const uint16_t* X = static_cast<const uint16_t*>(X_bf16);
 
-    // reference output Y = X W^T (fp32 accumulation), a plain library GEMM
-    const float one = 1.0f, zero = 0.0f;
-    if (cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, (int)d_out, (int)T, (int)d_in, &one, W, CUDA_R_16BF, (int)d_in, X,
-                     CUDA_R_16BF, (int)d_in, &zero, Yref, CUDA_R_32F, (int)d_out, CUBLAS_COMPUTE_32F,
-                     CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-        return WQ_ERR_CUDA;
+    // reference output Y = X W^T (fp32 accumulation), a plain library GEMM; the
+    // per-device handle is shared, so its stream is set and the GEMM enqueued
+    // under one lock
+    {
+        std::lock_guard<std::mutex> lk(g_blas_mu);
+        if (!g_blas[st.dev] && cublasCreate(&g_blas[st.dev]) != CUBLAS_STATUS_SUCCESS) return WQ_ERR_CUDA;
+        cublasHandle_t h = g_blas[st.dev];
+        const float one = 1.0f, zero = 0.0f;
+        if (cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS ||
+            cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, (int)d_out, (int)T, (int)d_in, &one, W, CUDA_R_16BF,
+                         (int)d_in, X, CUDA_R_16BF, (int)d_in, &zero, Yref, CUDA_R_32F, (int)d_out,
+                         CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+            return WQ_ERR_CUDA;
+    }
     cudaError_t e = launch_awq_colstats(X, T, d_in, lnm, mean_ln, s);
     for (int i = 0; e == cudaSuccess && i < kAwqAlphas; ++i) {
         e = launch_awq_scale_apply(W, d_out, X, T, d_in, lnm, mean_ln, i, nullptr, sbuf, Wp, Xp, st.num_sms, s);
