@@ -742,6 +742,24 @@ cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_s
     // 7.0 vs 9.0 us at 4096x4096, 14.7 vs 18.4 us at 11008x4096); longer rows and
     // M = 2 run faster on the tensor-memory kernel (15.7 vs 17.6 us at 4096x11008,
     // M = 2: 9.1 vs 10.6 us at 4096x4096).
+    if (base.M <= 8 && !gemv_ksplit_disabled()) {
+        KsArgs k = {};
+        k.X = base.X;
+        k.scales = base.scales;
+        k.zeros = base.zeros;
+        k.Y = base.Y;
+        k.status = base.status;
+        k.M = base.M;
+        k.N = base.N;
+        k.K = base.K;
+        k.G = base.G;
+        k.g = base.g;
+        k.g_shift = base.g_shift;
+        k.symmetric = base.symmetric;
+        k.y_fp32 = base.y_fp32;
+        const cudaError_t e = launch_gemv_ksplit(qweight, k, num_sms, opt, stream);
+        if (e != cudaErrorNotSupported) return e;
+    }
     const bool m1_first = base.M == 1 && base.K < 8192;
     if (m1_first) {
         const cudaError_t e = launch_gemv_m1(qweight, base, num_sms, opt, stream);

@@ -225,6 +225,11 @@ __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gsrc, 
         : "memory");
 }
 
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
@@ -250,6 +255,20 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
 }
 __device__ __forceinline__ void named_arrive(int id, int nthreads) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Copies of kernel parameters pinned in registers where they are taken (a
+// volatile move is not re-materialised later from the parameter bank).
+__device__ __forceinline__ int pin_i32(int v) {
+    int r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+    return r;
+}
+template <typename T>
+__device__ __forceinline__ T* pin_ptr(T* p) {
+    uint64_t r;
+    asm volatile("mov.b64 %0, %1;" : "=l"(r) : "l"(reinterpret_cast<uint64_t>(p)));
+    return reinterpret_cast<T*>(r);
 }
 
 __device__ __forceinline__ uint16_t ld_nc_u16(const uint16_t* p) {

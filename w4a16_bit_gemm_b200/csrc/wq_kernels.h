@@ -53,6 +53,27 @@ struct LaunchOptions {
 cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_sms, const LaunchOptions& opt,
                         cudaStream_t stream);
 
+// Decode GEMV for M <= 8 whose MMA tiles mix rows and k ranges (gemv_ksplit.cu);
+// two CTAs per SM when they fit, so consecutive launches overlap.
+struct KsArgs {
+    const void* X;           // bf16 [M][K]
+    const uint16_t* scales;  // fp16 [N][G]
+    const uint16_t* zeros;   // fp16 [N][G] or nullptr (symmetric)
+    void* Y;                 // [M][N] bf16 or fp32
+    uint32_t* status;
+    int M, N, K, G, g;
+    int g_shift;     // log2(g) when g is a power of two, else -1
+    int R;           // rows per CTA (set by the launcher)
+    int RC;          // rows per chunk (set by the launcher)
+    int nslots;      // shared-memory slots (set by the launcher)
+    int slot_bytes;  // (set by the launcher)
+    int symmetric;
+    int y_fp32;
+};
+
+cudaError_t launch_gemv_ksplit(const uint32_t* qweight, const KsArgs& a, int num_sms, const LaunchOptions& opt,
+                               cudaStream_t stream);
+
 // M <= 2 on tensor cores (dequantized weights as the A operand in tensor
 // memory); cudaErrorNotSupported for shapes it does not take.
 cudaError_t launch_gemv_tc(const uint32_t* qweight, const GemvArgs& a, int num_sms, const LaunchOptions& opt,
@@ -61,6 +82,8 @@ cudaError_t launch_gemv_tc(const uint32_t* qweight, const GemvArgs& a, int num_s
 // WQ_GEMV_TC=0 in the environment keeps M <= 2 off the tensor-memory kernel
 // (read once per process).
 bool gemv_tc_disabled();
+// WQ_GEMV_KSPLIT=0 keeps M <= 8 off the k-split kernel (read once per process).
+bool gemv_ksplit_disabled();
 
 // Prefill GEMM on tcgen05 tensor cores, any M (used for M > 16).
 struct GemmArgs {
