@@ -122,6 +122,10 @@ def _load(path: str | None = None):
             lib.wqo_awq_search.restype = i32
             lib.wqo_awq_scales.argtypes = [P, i64, i64, ctypes.c_double, P]
             lib.wqo_awq_scales.restype = None
+            lib.wqo_ln_f64.argtypes = [ctypes.c_double]
+            lib.wqo_ln_f64.restype = ctypes.c_double
+            lib.wqo_exp_f64.argtypes = [ctypes.c_double]
+            lib.wqo_exp_f64.restype = ctypes.c_double
             lib.wqo_pack8.argtypes = [P, i64, i64, P]
             lib.wqo_pack8.restype = i32
             lib.wqo_unpack8.argtypes = [P, i64, i64, P]
@@ -309,6 +313,16 @@ def awq_search(W_bits: np.ndarray, X_bits: np.ndarray, group_size: int = 128, sy
     if rc != 0:
         raise ValueError("oracle AWQ search rejected its arguments")
     return codes, scales, zeros, s, losses, int(best.value)
+
+
+def ln_f64(x: float) -> float:
+    """ln x by the fixed fp64 procedure of the AWQ scales (x positive, normal)."""
+    return _load().wqo_ln_f64(float(x))
+
+
+def exp_f64(x: float) -> float:
+    """e^x by the fixed fp64 procedure of the AWQ scales (|x| < 700)."""
+    return _load().wqo_exp_f64(float(x))
 
 
 def awq_scales(X_bits: np.ndarray, alpha: float) -> np.ndarray:

@@ -508,6 +508,8 @@ int wqo_quantize_clip(const uint16_t* W, int64_t d_out, int64_t d_in, int64_t g,
 /*  - s_j = bf16_rn(fl32(exp(alpha (ln m_j - mean_j ln m_j)))), i.e. m^alpha  */
 /*    over its geometric mean (fp64), rounded to fp32 then bf16, so that the  */
 /*    two products below are one multiply or divide and one rounding each;    */
+/*    ln and exp are wqo_ln_f64 / wqo_exp_f64 below (a fixed fp64 procedure), */
+/*    the mean of ln m is summed in channel order;                            */
 /*  - W'[n,j] = bf16_rn(fl32(W[n,j] s_j)); X'[t,j] = bf16_rn(fl32(X[t,j]/s_j)); */
 /*  - Q(W') is the RTN artifact of W' (quantize_group) and its dequant;        */
 /*  - loss = sum_{t,n} (Y[t,n] - Y'[t,n])^2 with Y = X W^T and Y' = X' Q(W')^T  */
@@ -516,6 +518,64 @@ int wqo_quantize_clip(const uint16_t* W, int64_t d_out, int64_t d_in, int64_t g,
 /* ------------------------------------------------------------------------ */
 
 #define WQO_AWQ_ALPHAS 11
+
+/* ln and exp of the AWQ scales, as one fixed sequence of IEEE binary64       */
+/* operations (each multiply, add, subtract and divide rounded on its own, no */
+/* fused multiply-add: this file is compiled with -ffp-contract=off), so that */
+/* any implementation that follows the same steps obtains the same bits; the  */
+/* pages give the formula s = m^alpha / geomean but no evaluation procedure.  */
+/* Both use the argument reduction of W. J. Cody and W. Waite, "Software      */
+/* Manual for the Elementary Functions" (1980): ln 2 split into a head with   */
+/* 21 trailing zero bits (k ln2_hi exact for |k| < 2^21) and a tail.          */
+static const double WQO_LN2_HI = 0x1.62e42fee00000p-1;
+static const double WQO_LN2_LO = 0x1.a39ef35793c76p-33;
+static const double WQO_INV_LN2 = 0x1.71547652b82fep+0;
+static const double WQO_SQRT2 = 0x1.6a09e667f3bcdp+0;
+
+/* ln x for a positive normal x: x = f 2^e with f in [sqrt(2)/2, sqrt(2)),     */
+/* u = (f - 1) / (f + 1), ln f = 2 atanh u = 2 u (1 + u^2/3 + u^4/5 + ...),    */
+/* twelve terms (|u| <= 0.1716, the first dropped term is below 2^-60),       */
+/* evaluated by Horner's rule in u^2; ln x = e ln2_hi + (e ln2_lo + ln f).     */
+double wqo_ln_f64(double x) {
+    uint64_t b;
+    memcpy(&b, &x, 8);
+    int e = (int)((b >> 52) & 0x7ff) - 1023;
+    const uint64_t fb = (b & 0x000fffffffffffffull) | 0x3ff0000000000000ull;
+    double f;
+    memcpy(&f, &fb, 8);
+    if (f > WQO_SQRT2) {
+        f = f * 0.5;
+        e += 1;
+    }
+    const double u = (f - 1.0) / (f + 1.0);
+    const double v = u * u;
+    double p = 1.0 / 23.0;
+    for (int k = 10; k >= 0; --k) p = p * v + 1.0 / (double)(2 * k + 1);
+    const double lnf = (u + u) * p;
+    const double de = (double)e;
+    return de * WQO_LN2_HI + (de * WQO_LN2_LO + lnf);
+}
+
+/* e^x for |x| < 700: k = rint(x / ln 2) (round half to even, by adding and   */
+/* subtracting 1.5 2^52), r = (x - k ln2_hi) - k ln2_lo, e^r by its Taylor    */
+/* polynomial of degree 13 (|r| <= 0.347, the first dropped term below 2^-57) */
+/* in Horner form with coefficients 1/i!, then the exact product by 2^k.      */
+double wqo_exp_f64(double x) {
+    const double magic = 0x1.8p52;
+    const double kd = (x * WQO_INV_LN2 + magic) - magic;
+    const double r = (x - kd * WQO_LN2_HI) - kd * WQO_LN2_LO;
+    double fact = 1.0;
+    for (int i = 2; i <= 13; ++i) fact *= (double)i;  /* 13!, exact */
+    double p = 1.0 / fact;
+    for (int i = 12; i >= 0; --i) {
+        fact /= (double)(i + 1);                       /* i!, exact */
+        p = p * r + 1.0 / fact;
+    }
+    const uint64_t sb = (uint64_t)((int64_t)kd + 1023) << 52;
+    double scale;
+    memcpy(&scale, &sb, 8);
+    return p * scale;
+}
 
 int wqo_dequantize(const int32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,
                    int64_t d_in, int64_t g, uint16_t* W_hat, int nthreads);
@@ -554,15 +614,15 @@ void wqo_awq_scales(const uint16_t* X, int64_t T, int64_t K, double alpha, uint1
         for (int64_t t = 0; t < T; ++t) acc += fabs((double)wqo_bf16_to_f32(X[t * K + j]));
         double m = acc / (double)T;
         if (m < 0x1p-30) m = 0x1p-30;
-        lnm[j] = log(m);
+        lnm[j] = wqo_ln_f64(m);
     }
     for (int64_t j = 0; j < K; ++j) mean_ln += lnm[j];
     mean_ln /= (double)K;
     for (int64_t j = 0; j < K; ++j) {
 #if WQO_MUTANT == 11 /* mistake: scales inverted (divide instead of multiply) */
-        s_out[j] = wqo_f32_to_bf16((float)exp(-alpha * (lnm[j] - mean_ln)));
+        s_out[j] = wqo_f32_to_bf16((float)wqo_exp_f64(-alpha * (lnm[j] - mean_ln)));
 #else
-        s_out[j] = wqo_f32_to_bf16((float)exp(alpha * (lnm[j] - mean_ln)));
+        s_out[j] = wqo_f32_to_bf16((float)wqo_exp_f64(alpha * (lnm[j] - mean_ln)));
 #endif
     }
     free(lnm);

@@ -116,3 +116,43 @@ def test_scale_migration_identity():
     Y = vals(Xb) @ vals(Wb).T
     Y2 = (vals(Xb) / s[None, :]) @ (vals(Wb) * s[None, :]).T
     assert np.allclose(Y, Y2, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# The fixed fp64 ln / exp of the scales (Cody-Waite reduction; atanh series,
+# Taylor polynomial): pinned to the libm functions, to closed forms and to
+# their own inverse relation.
+# ---------------------------------------------------------------------------
+
+def _ulps(a, b):
+    return abs(a - b) / np.spacing(abs(b)) if b != 0 else abs(a) / np.spacing(0.0)
+
+
+def test_ln_matches_libm_within_two_ulps():
+    import math
+    rng = np.random.default_rng(31)
+    xs = np.concatenate([np.exp(rng.uniform(-30, 30, 5000)), rng.uniform(0.5, 2.0, 2000),
+                         [2.0 ** -30, 1.0 - 2 ** -52, 1.0 + 2 ** -52, np.sqrt(2.0), 1e-9, 123456.789]])
+    worst = max(_ulps(oracle.ln_f64(x), math.log(x)) for x in xs)
+    assert worst <= 2.0, worst
+
+
+def test_exp_matches_libm_within_two_ulps():
+    import math
+    rng = np.random.default_rng(32)
+    xs = np.concatenate([rng.uniform(-40, 40, 5000), rng.uniform(-0.35, 0.35, 2000),
+                         [0.5 * math.log(2.0), -0.5 * math.log(2.0), 1e-12, -20.5]])
+    worst = max(_ulps(oracle.exp_f64(x), math.exp(x)) for x in xs)
+    assert worst <= 2.0, worst
+
+
+def test_ln_exp_closed_forms():
+    import math
+    assert oracle.ln_f64(1.0) == 0.0
+    assert oracle.exp_f64(0.0) == 1.0
+    for k in range(-30, 31):
+        if k:  # ln 2^k = k ln 2 (k ln2_hi is exact, so only the tail rounds)
+            assert _ulps(oracle.ln_f64(2.0 ** k), k * math.log(2.0)) <= 1.0
+    # e^(ln x) = x to a few ulps, across the range the scales use
+    for x in (1e-6, 0.02, 0.8, 1.0, 3.0, 50.0, 1e5):
+        assert _ulps(oracle.exp_f64(oracle.ln_f64(x)), x) <= 8.0
