@@ -18,13 +18,12 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - All array arguments are DEVICE pointers owned by the caller.  The library
- *   never frees or retains them.  The library owns one device status word per
- *   device (a static device variable) and, only once wq_awq_search_static is
- *   called, that function's static scratch array; wq_awq_search's reference
- *   GEMM runs in cuBLAS, which allocates its own workspace on first use.  No
- *   other entry point allocates device memory.  The first call on a device
- *   looks up the status word's address and should not be made inside a
- *   stream capture.
+ *   never frees or retains them.  It owns one device status word per device
+ *   (a static device variable) and the static scratch array of
+ *   wq_awq_search_static (a static device variable in its own module).  No
+ *   entry point allocates device memory, and no other library is called on
+ *   the device path.  The first call on a device looks up the status word's
+ *   address and should not be made inside a stream capture.
  * - Matrices are dense row-major.  bf16 and fp16 values are passed as their
  *   16-bit storage (void*).
  * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
@@ -208,10 +207,15 @@ size_t wq_linear_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in);
  *   for alpha_i = i / 10, i = 0..10:
  *     s_j  = bf16_rn(fl32(exp(alpha_i (ln m_j - mean_j ln m_j))))
  *            (mean|x|^alpha divided by its geometric mean over the channels);
+ *            ln and exp are one fixed sequence of IEEE fp64 operations
+ *            (Cody-Waite reduction by ln 2; the atanh series for ln, a
+ *            degree-13 Taylor polynomial for exp; no fused multiply-add) and
+ *            the mean is summed in channel order, so s is reproducible bit
+ *            for bit by any implementation of the same steps;
  *     W'   = bf16_rn(fl32(W[n][j] s_j)),  X' = bf16_rn(fl32(X[t][j] / s_j));
  *     Q(W') = the wq_quantize_rtn artifact of W';
  *     loss_i = sum_{t,n} (Y[t][n] - Y'[t][n])^2 in fp64, with Y = X W^T
- *            (fp32 accumulation, a library GEMM) and Y' = X' Q(W')^T from
+ *            (fp32 accumulation, the tcgen05 GEMM on bf16 W) and Y' = X' Q(W')^T from
  *            wq_linear_w4a16 with fp32 output;
  *   the smallest loss is kept (ties: the smaller i).  alpha_0 = 0 gives s = 1,
  *   i.e. plain RTN.  The losses are deterministic run to run.
@@ -231,7 +235,7 @@ size_t wq_linear_workspace_bytes(int64_t M, int64_t d_out, int64_t d_in);
  *               bytes, 256-byte aligned, owned by the caller.
  * All work is queued on `stream`; the call does not synchronize.
  * Errors: WQ_ERR_INVALID_ARG as wq_quantize_rtn plus a missing or small
- * workspace or a bad T; WQ_ERR_CUDA if a launch or the library GEMM fails.
+ * workspace, a bad T or d_in not a multiple of 8; WQ_ERR_CUDA if a launch fails.
  * Device flags: as wq_quantize_rtn, from every candidate's quantization.
  */
 wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const void* X_bf16, int64_t T,
@@ -243,13 +247,24 @@ wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const v
 size_t wq_awq_workspace_bytes(int64_t d_out, int64_t d_in, int64_t T, int32_t group_size);
 
 /*
- * wq_awq_search_static -- wq_awq_search without a caller workspace: the
- * scratch is a device array owned by the library (wq_awq_static_scratch_bytes()
- * bytes, reserved on a device when a process first calls this function).
+ * wq_awq_search_static -- wq_awq_search without a caller workspace, for
+ * callers that cannot allocate device memory themselves: code running under
+ * a host allocator it may not bypass (a framework's caching allocator, a
+ * memory pool sized at start-up), or a process that must not grow its device
+ * footprint after start-up.  This paper has no counterpart; the scratch is a
+ * file-scope device array owned by the library (wq_awq_static_scratch_bytes()
+ * = 80 MiB, enough for a 4096 x 4096 layer with 512 calibration tokens).  It
+ * is reserved when the CUDA module holding it is loaded on a device: at this
+ * function's first call under lazy module loading (the default), at context
+ * creation under CUDA_MODULE_LOADING=EAGER; it stays reserved until the
+ * process exits.  The call allocates nothing (no cudaMalloc, no library
+ * workspace).  Its first call on a device looks up the array's address and
+ * should come before any stream capture.
  * Arguments, results and errors as wq_awq_search, plus WQ_ERR_UNSUPPORTED
  * when wq_awq_workspace_bytes(d_out, d_in, T, group_size) exceeds the array.
- * All calls on a device share the array: they must not overlap in time
- * (queue them on one stream).
+ * Every call on a device shares the array and leaves its contents behind
+ * (each search writes every part it reads first): calls whose work overlaps
+ * on the GPU race, so queue them on one stream or otherwise serialize them.
  */
 wq_status wq_awq_search_static(const void* W_bf16, int64_t d_out, int64_t d_in, const void* X_bf16,
                                int64_t T, int32_t group_size, int32_t symmetric, uint32_t* qweight,

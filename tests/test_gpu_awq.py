@@ -3,15 +3,15 @@ oracle ("Quantization Algorithms" study notes, AWQ procedure).
 
 What must agree and how:
   - the 11 losses: the oracle sums in fp64 over fp64 outputs, the library over
-    fp32 outputs (a library GEMM for X W^T, the W4A16 linear for X' Q(W')^T),
-    so they agree to a relative 1e-4 (the fp32 output rounding is ~1e-7 of |Y|
-    against a quantization error of a few per cent of |Y|);
-  - the kept alpha: the oracle's argmin, unless the oracle's own losses at the
-    two choices are within that tolerance (either is then correct);
-  - s: the oracle's scales for the kept alpha, bit for bit except for at most a
-    few channels one bf16 ulp apart (exp/log of two libraries near a rounding
-    boundary);
-  - the artifact: bit-exact against the oracle RTN of bf16(W s_gpu)."""
+    fp32 outputs (the tcgen05 GEMM on bf16 W for X W^T, the W4A16 linear for
+    X' Q(W')^T), so they agree to a relative 1e-4 (the fp32 output rounding is
+    ~1e-7 of |Y| against a quantization error of a few per cent of |Y|);
+  - the kept alpha: equal to the oracle's (every case here has a loss gap far
+    above that tolerance);
+  - s: the oracle's scales for the kept alpha, bit for bit (both sides evaluate
+    ln and exp by the same fixed fp64 procedure and sum the mean of ln m in
+    channel order);
+  - the artifact: bit-exact against the oracle's own search."""
 import numpy as np
 import pytest
 import torch
@@ -63,23 +63,16 @@ def check(W, X, g=128, sym=False):
     oc, osc, oz, os_, olosses, obest = oracle.awq_search(Wb, Xb, g, symmetric=sym)
     # losses
     assert np.all(np.abs(losses - olosses) <= LOSS_RTOL * olosses + 1e-30), (losses, olosses)
-    # the kept alpha
-    if best != obest:
-        assert olosses[best] - olosses[obest] <= LOSS_RTOL * olosses[obest], (best, obest, olosses)
-    assert losses[best] == losses.min()
-    assert best == int(np.argmin(losses))
-    # scales of the kept alpha
-    s_ref = oracle.awq_scales(Xb, best / 10.0) if best != obest else os_
-    d = np.abs(s_gpu.astype(np.int32) - s_ref.astype(np.int32))
-    assert d.max() <= 1 and int((d != 0).sum()) <= max(2, s_gpu.size // 1000)
-    # artifact: RTN of bf16(W s_gpu), bit-exact
-    rq, rs, rz, rf, _ = oracle.quantize_pack4(scaled_weight_bits(Wb, s_gpu), g, sym)
-    assert np.array_equal(bits32(r.packed.qweight), rq)
-    assert np.array_equal(bits16(r.packed.scales), rs)
+    # the kept alpha, and a gap that makes it the only correct answer
+    assert best == obest, (best, obest, olosses)
+    others = np.delete(olosses, obest)
+    assert np.all(others - olosses[obest] > LOSS_RTOL * olosses[obest]) or np.all(olosses == olosses[0])
+    # the scales of the kept alpha and the artifact, bit for bit
+    assert np.array_equal(s_gpu, os_)
+    assert np.array_equal(oracle.unpack4(bits32(r.packed.qweight), W.shape[1], sym), oc)
+    assert np.array_equal(bits16(r.packed.scales), osc)
     if not sym:
-        assert np.array_equal(bits16(r.packed.zeros), rz)
-    if best == obest and np.array_equal(s_gpu, os_):
-        assert np.array_equal(oracle.unpack4(rq, W.shape[1], sym), oc)
+        assert np.array_equal(bits16(r.packed.zeros), oz)
     return r, losses, best, olosses, obest
 
 
@@ -176,11 +169,13 @@ def test_awq_layer_output_through_the_linear():
 
 def test_awq_full_size_attention_projection():
     """4096 x 4096 with 512 calibration tokens (the bench workload): the
-    oracle is too slow for the whole search, so check what holds at any size.
-    s equals the oracle's scales for the kept alpha (to an ulp); the artifact is
-    the (oracle-parity-tested) RTN of bf16(W s) bit for bit; two of the losses
-    are recomputed in fp64 on the device with torch from artifacts that the
-    RTN entry point produces."""
+    oracle's whole search is too slow here, so its pieces are used.
+    - s equals the oracle's scales for the kept alpha, bit for bit;
+    - the artifact equals the oracle's RTN of bf16(W s) with the oracle's s;
+    - the losses of alpha = 0 and the kept alpha, recomputed in fp64 from the
+      oracle's artifacts (torch fp64 products), agree to LOSS_RTOL;
+    - the runner-up loss is more than 3 LOSS_RTOL above the kept one, so any
+      loss computation within that tolerance keeps the same alpha."""
     b = _b()
     W = syn.case_weight(syn.ATTN, 0, "cpu")
     X = syn.activations(512, 4096, 21, 2, "cpu", channel_outlier_frac=0.001)
@@ -191,20 +186,22 @@ def test_awq_full_size_attention_projection():
     best = int(r.best.item())
     losses = r.losses.cpu().numpy()
     assert best == int(np.argmin(losses)) and best > 0
-    s_gpu = bits16(r.s)
-    s_ref = oracle.awq_scales(bits16(X), best / 10.0)
-    d = np.abs(s_gpu.astype(np.int32) - s_ref.astype(np.int32))
-    assert d.max() <= 1 and int((d != 0).sum()) <= 4
-    Wp_bits = scaled_weight_bits(bits16(W), s_gpu)
-    Wp = torch.from_numpy(Wp_bits.view(np.int16)).view(torch.bfloat16).cuda()
-    p = b.quantize_rtn(Wp)
-    assert torch.equal(p.qweight, r.packed.qweight) and torch.equal(p.scales, r.packed.scales)
-    assert torch.equal(p.zeros, r.packed.zeros)
+    gaps = np.delete(losses, best) - losses[best]
+    assert gaps.min() > 3 * LOSS_RTOL * losses[best], (losses, best)
+    Wb, Xb = bits16(W), bits16(X)
+    s_ref = oracle.awq_scales(Xb, best / 10.0)
+    assert np.array_equal(bits16(r.s), s_ref)
+    rq, rs, rz, _, _ = oracle.quantize_pack4(scaled_weight_bits(Wb, s_ref), 128, False)
+    assert np.array_equal(bits32(r.packed.qweight), rq)
+    assert np.array_equal(bits16(r.packed.scales), rs) and np.array_equal(bits16(r.packed.zeros), rz)
     Y = Xd.double() @ Wd.double().T
+    X32 = f64_from_bf16_bits(Xb).astype(np.float32)
     for i in (0, best):
-        si = torch.from_numpy(oracle.awq_scales(bits16(X), i / 10.0).view(np.int16)).view(torch.bfloat16).cuda()
-        pi = b.quantize_rtn((Wd.float() * si.float()).to(torch.bfloat16))
-        Xi = b.awq_scale_activations(Xd, si)
-        Yi = Xi.double() @ b.dequantize(pi).double().T
+        si = oracle.awq_scales(Xb, i / 10.0)
+        q, sc, z, _, codes = oracle.quantize_pack4(scaled_weight_bits(Wb, si), 128, False)
+        Wh = f64_from_bf16_bits(oracle.dequantize(codes, sc, z, 128))
+        s32 = f64_from_bf16_bits(si).astype(np.float32)
+        Xi = f64_from_bf16_bits(bits16(torch.from_numpy((X32 / s32[None, :]).astype(np.float32)).to(torch.bfloat16)))
+        Yi = torch.from_numpy(Xi).cuda() @ torch.from_numpy(Wh).cuda().T
         li = float(((Y - Yi) ** 2).sum())
         assert abs(losses[i] - li) <= LOSS_RTOL * li, (i, losses[i], li)

@@ -3,8 +3,8 @@
     python -m w4a16_bit_gemm_b200.build [--verbose-ptxas] [--force]
 
 Each .cu file under csrc/ is compiled to an object file in _build/ and linked
-into w4a16_bit_gemm_b200/libwq.so (CUDA runtime linked statically; cuBLAS
-dynamically, for the full-precision reference GEMM of the AWQ search).
+into w4a16_bit_gemm_b200/libwq.so (CUDA runtime linked statically; no other
+library).
 """
 from __future__ import annotations
 
@@ -78,8 +78,7 @@ def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = False)
         raise RuntimeError("nvcc failed")
     if force or jobs or _stale(LIB, objs):
         tmp = LIB + ".tmp%d" % os.getpid()
-        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-lcublas",
-               "-Xlinker", "-rpath," + CUDA_LIB]
+        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)

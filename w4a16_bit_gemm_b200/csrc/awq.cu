@@ -7,7 +7,9 @@
 // kernels compute the statistics, the scales, W' and X', and the losses:
 //  - m_j = (sum_t |X[t,j]|) / T in fp64 (an exact sum of bf16 values, so the
 //    summation order does not matter), floored at 2^-30, kept as ln m_j;
-//  - s_j = bf16_rn(fl32(exp(alpha (ln m_j - mean_j ln m_j))));
+//  - s_j = bf16_rn(fl32(exp(alpha (ln m_j - mean_j ln m_j)))), with ln and exp
+//    evaluated by one fixed sequence of IEEE fp64 operations (below) and the
+//    mean summed in channel order, so the scales are reproducible bit for bit;
 //  - W'[n,j] = bf16_rn(fl32(W[n,j] s_j)), X'[t,j] = bf16_rn(fl32(X[t,j] / s_j));
 //  - loss = sum (Y_ref - Y')^2 in fp64 over fp32 outputs, reduced in a fixed
 //    order (deterministic).
@@ -24,6 +26,55 @@ constexpr int kAwqThreads = 256;
 constexpr int kAwqReduceThreads = 1024;
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// ln and exp as fixed sequences of IEEE binary64 operations: every product,
+// sum and quotient rounded on its own through the _rn intrinsics (no fused
+// multiply-add), with the argument reduction of W. J. Cody and W. Waite,
+// "Software Manual for the Elementary Functions" (1980): ln 2 as a head with 21
+// trailing zero bits (k * head exact for |k| < 2^21) plus a tail.
+constexpr double kLn2Hi = 0x1.62e42fee00000p-1;
+constexpr double kLn2Lo = 0x1.a39ef35793c76p-33;
+constexpr double kInvLn2 = 0x1.71547652b82fep+0;
+constexpr double kSqrt2 = 0x1.6a09e667f3bcdp+0;
+
+// ln x, x positive and normal: x = f 2^e with f in [sqrt(2)/2, sqrt(2));
+// ln f = 2 atanh(u), u = (f - 1) / (f + 1), as 2 u times the series
+// sum_{k=0}^{11} u^(2k) / (2k + 1) in Horner form (|u| <= 0.1716);
+// ln x = e ln2_hi + (e ln2_lo + ln f).
+__device__ double awq_ln(double x) {
+    const unsigned long long b = (unsigned long long)__double_as_longlong(x);
+    int e = (int)((b >> 52) & 0x7ffull) - 1023;
+    double f = __longlong_as_double((long long)((b & 0x000fffffffffffffull) | 0x3ff0000000000000ull));
+    if (f > kSqrt2) {
+        f = __dmul_rn(f, 0.5);
+        e += 1;
+    }
+    const double u = __ddiv_rn(__dsub_rn(f, 1.0), __dadd_rn(f, 1.0));
+    const double v = __dmul_rn(u, u);
+    double p = __ddiv_rn(1.0, 23.0);
+    for (int k = 10; k >= 0; --k) p = __dadd_rn(__dmul_rn(p, v), __ddiv_rn(1.0, (double)(2 * k + 1)));
+    const double lnf = __dmul_rn(__dadd_rn(u, u), p);
+    const double de = (double)e;
+    return __dadd_rn(__dmul_rn(de, kLn2Hi), __dadd_rn(__dmul_rn(de, kLn2Lo), lnf));
+}
+
+// e^x, |x| < 700: k = rint(x / ln 2) (half to even: add and subtract 1.5 2^52),
+// r = (x - k ln2_hi) - k ln2_lo, e^r by its degree-13 Taylor polynomial
+// (coefficients 1/i!, Horner form, |r| <= 0.347), times 2^k (exact).
+__device__ double awq_exp(double x) {
+    const double magic = 0x1.8p52;
+    const double kd = __dsub_rn(__dadd_rn(__dmul_rn(x, kInvLn2), magic), magic);
+    const double r = __dsub_rn(__dsub_rn(x, __dmul_rn(kd, kLn2Hi)), __dmul_rn(kd, kLn2Lo));
+    double fact = 1.0;
+    for (int i = 2; i <= 13; ++i) fact = __dmul_rn(fact, (double)i);  // 13!
+    double p = __ddiv_rn(1.0, fact);
+    for (int i = 12; i >= 0; --i) {
+        fact = __ddiv_rn(fact, (double)(i + 1));  // i!, exact
+        p = __dadd_rn(__dmul_rn(p, r), __ddiv_rn(1.0, fact));
+    }
+    const double scale = __longlong_as_double((long long)(((unsigned long long)((long long)kd + 1023)) << 52));
+    return __dmul_rn(p, scale);
+}
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
@@ -33,25 +84,18 @@ __global__ void __launch_bounds__(kAwqThreads) awq_colstats_kernel(const uint16_
     const int64_t j = (int64_t)blockIdx.x * kAwqThreads + threadIdx.x;
     if (j >= K) return;
     double acc = 0.0;
-    for (int64_t t = 0; t < T; ++t) acc += fabs((double)bf16_bits_to_f32(X[t * K + j]));
-    double m = acc / (double)T;
+    for (int64_t t = 0; t < T; ++t) acc = __dadd_rn(acc, fabs((double)bf16_bits_to_f32(X[t * K + j])));
+    double m = __ddiv_rn(acc, (double)T);
     if (m < 0x1p-30) m = 0x1p-30;
-    lnm[j] = log(m);
+    lnm[j] = awq_ln(m);
 }
 
-// One block: mean of v[0..n) in a fixed order (strided per-thread sums, then a tree).
-__global__ void __launch_bounds__(kAwqReduceThreads) awq_mean_kernel(const double* __restrict__ v, int64_t n,
-                                                                     double* __restrict__ out) {
-    __shared__ double part[kAwqReduceThreads];
+// Mean of v[0..n), summed in index order by one thread (once per search).
+__global__ void awq_mean_kernel(const double* __restrict__ v, int64_t n, double* __restrict__ out) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
     double acc = 0.0;
-    for (int64_t i = threadIdx.x; i < n; i += kAwqReduceThreads) acc += v[i];
-    part[threadIdx.x] = acc;
-    __syncthreads();
-    for (int w = kAwqReduceThreads / 2; w > 0; w >>= 1) {
-        if ((int)threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) *out = part[0] / (double)n;
+    for (int64_t i = 0; i < n; ++i) acc = __dadd_rn(acc, v[i]);
+    *out = __ddiv_rn(acc, (double)n);
 }
 
 // s for alpha = i / 10, with i = *best if best is given, else alpha_idx.
@@ -62,8 +106,8 @@ __global__ void __launch_bounds__(kAwqThreads) awq_scales_kernel(const double* _
     const int64_t j = (int64_t)blockIdx.x * kAwqThreads + threadIdx.x;
     if (j >= K) return;
     const int i = best ? *best : alpha_idx;
-    const double alpha = (double)i / 10.0;
-    s[j] = f32_to_bf16_bits(__double2float_rn(exp(alpha * (lnm[j] - *mean_ln))));
+    const double alpha = __ddiv_rn((double)i, 10.0);
+    s[j] = f32_to_bf16_bits(__double2float_rn(awq_exp(__dmul_rn(alpha, __dsub_rn(lnm[j], *mean_ln)))));
 }
 
 // W' = bf16(W s) for n_w rows, X' = bf16(X / s) for n_x rows; 8 weights per thread.
@@ -146,7 +190,7 @@ constexpr int kAwqLossBlocks = 296;
 cudaError_t launch_awq_colstats(const uint16_t* X, int64_t T, int64_t K, double* lnm, double* mean_ln,
                                 cudaStream_t stream) {
     awq_colstats_kernel<<<(unsigned)((K + kAwqThreads - 1) / kAwqThreads), kAwqThreads, 0, stream>>>(X, T, K, lnm);
-    awq_mean_kernel<<<1, kAwqReduceThreads, 0, stream>>>(lnm, K, mean_ln);
+    awq_mean_kernel<<<1, 32, 0, stream>>>(lnm, K, mean_ln);
     return cudaGetLastError();
 }
 

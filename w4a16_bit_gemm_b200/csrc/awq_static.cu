@@ -1,10 +1,14 @@
 // awq_static.cu -- the AWQ scaling search with library-owned scratch.
 //
 // wq_awq_search_static runs wq_awq_search on a file-scope device array
-// instead of a caller workspace.  The array lives in this translation unit's
-// own module, so its device memory is reserved only once a process calls
-// this entry point.  Every call on a device shares the array: calls must not
-// overlap in time (queue them on one stream).
+// instead of a caller workspace, for callers that cannot allocate device
+// memory (they run under an allocator they may not bypass, or must not grow
+// their device footprint after start-up); the search itself allocates
+// nothing.  The array is reserved when the CUDA module holding it is loaded
+// on a device: at the first call under lazy module loading (the default), at
+// context creation under CUDA_MODULE_LOADING=EAGER.  Every call on a device
+// shares the array: calls whose work overlaps on the GPU race (queue them on
+// one stream).
 #include <cuda_runtime.h>
 #include <stdint.h>
 

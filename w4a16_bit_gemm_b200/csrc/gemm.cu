@@ -20,6 +20,10 @@
 // Barriers: full1/empty1 (ring 1: TMA bytes; MMA commit + 8 producer warps),
 //           full2/empty2 (ring 2: 8 producer warps; MMA commit), acc (final
 //           MMA commit).  Every wait is bounded (WQ_DEVFLAG_TIMEOUT).
+// BITS = 16 is the same kernel on unquantized bf16 weights (the reference
+// product X W^T of the AWQ search): TMA writes the B tile [256 x 64] straight
+// into ring 1 in the SWIZZLE_128B K-major layout the dequant warps produce
+// otherwise, and warps 2-9 only run the epilogue.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -41,15 +45,15 @@ constexpr int kNumProducerWarps = 8;
 
 template <int MSUB, int BITS>
 struct GemmSmem {
-    // X / packed-W ring depth: 4, or 3 when 8-bit tiles would not fit
-    static constexpr int kS1 = (BITS == 8 && MSUB == 2) ? 3 : 4;
+    // X / packed-W ring depth: 4, or 3 when 8-bit or bf16 tiles would not fit
+    static constexpr int kS1 = ((BITS == 8 || BITS == 16) && MSUB == 2) ? 3 : 4;
     static constexpr int kATile = 128 * MSUB * kBK * 2;  // bytes
-    static constexpr int kWqTile = kBN * kBK * BITS / 8; // packed bytes
-    static constexpr int kBTile = kBN * kBK * 2;
+    static constexpr int kWqTile = kBN * kBK * BITS / 8; // packed bytes (bf16 B tile when BITS = 16)
+    static constexpr int kBTile = BITS == 16 ? 0 : kBN * kBK * 2;
     static constexpr int kStage1 = kATile + kWqTile;
     static constexpr int kOffA = 0;                           // S1 x A tiles
     static constexpr int kOffWq = kOffA + kS1 * kATile;       // S1 x packed tiles
-    static constexpr int kOffB = kOffWq + kS1 * kWqTile;      // S2 x B tiles
+    static constexpr int kOffB = kOffWq + kS1 * kWqTile;      // S2 x B tiles (none for bf16)
     static constexpr int kOffBar = kOffB + kS2 * kBTile;      // barriers
     static constexpr int kBytes = kOffBar + 256;
     static constexpr int kAlloc = kBytes + 1024;              // + alignment slack
@@ -82,7 +86,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kS1; ++s) {
             mbar_init(&full1[s], 1);
-            mbar_init(&empty1[s], 1 + kNumProducerWarps);
+            mbar_init(&empty1[s], BITS == 16 ? 1 : 1 + kNumProducerWarps);
         }
         for (int s = 0; s < kS2; ++s) {
             mbar_init(&full2[s], kNumProducerWarps);
@@ -119,7 +123,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                 for (int ms = 0; ms < MSUB; ++ms)
                     tma_load_2d(As + ms * (128 * kBK * 2), &tmap_x, &full1[s], kb * kBK, m0 + 128 * ms);
-                tma_load_2d(smem + SL::kOffWq + s * SL::kWqTile, &tmap_wq, &full1[s], kb * (kBK * BITS / 32), n0);
+                if constexpr (BITS == 16)
+                    tma_load_2d(smem + SL::kOffWq + s * SL::kWqTile, &tmap_wq, &full1[s], kb * kBK, n0);
+                else
+                    tma_load_2d(smem + SL::kOffWq + s * SL::kWqTile, &tmap_wq, &full1[s], kb * (kBK * BITS / 32), n0);
                 ++issued;
             }
             // drain: wait until the last load into every stage has landed
@@ -134,13 +141,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s1 = kb % kS1, s2 = kb % kS2;
                 if (!mbar_wait(&full1[s1], (uint32_t)(kb / kS1) & 1u, a.status) ||
-                    !mbar_wait(&full2[s2], (uint32_t)(kb / kS2) & 1u, a.status)) {
+                    (BITS != 16 && !mbar_wait(&full2[s2], (uint32_t)(kb / kS2) & 1u, a.status))) {
                     atomicExch(abort_flag, 1);
                     break;
                 }
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(smem + SL::kOffA + s1 * SL::kATile);
-                const uint32_t b_addr = smem_u32(smem + SL::kOffB + s2 * SL::kBTile);
+                const uint32_t b_addr = BITS == 16 ? smem_u32(smem + SL::kOffWq + s1 * SL::kWqTile)
+                                                   : smem_u32(smem + SL::kOffB + s2 * SL::kBTile);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk) {
                     const uint64_t bdesc = sw128_kmajor_desc(b_addr + kk * 32);
@@ -151,7 +159,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
                 tc_commit(&empty1[s1]);
-                tc_commit(&empty2[s2]);
+                if constexpr (BITS != 16) tc_commit(&empty2[s2]);
             }
             tc_commit(accbar);  // completes once every MMA issued above has finished
         }
@@ -163,14 +171,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool nvalid = n < a.N;
         const bool sym = a.symmetric != 0;
         const int kw = a.K * BITS / 32;  // packed words per row
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = 0; kb < (BITS == 16 ? 0 : nkb); ++kb) {
             const int s1 = kb % kS1, s2 = kb % kS2;
             if (__any_sync(0xffffffffu, *(volatile int*)abort_flag != 0)) break;
             // group constants for the two 32-k halves of this k block
             const int kbase = kb * kBK;
             const int gA = kbase / a.g, gB = (kbase + 32) / a.g;
             uint8_t* brow = smem + SL::kOffB + s2 * SL::kBTile + i * 128;
-            if constexpr (BITS == 4) {
+            if constexpr (BITS == 16) {
+                // no producer work: TMA loads the bf16 B tiles
+            } else if constexpr (BITS == 4) {
                 GroupConsts cA, cB;
                 if (nvalid) {
                     const int64_t ia = (int64_t)n * a.G + gA;
@@ -331,9 +341,13 @@ cudaError_t launch_gemm_bits(const GemmArgs& a, int num_sms, cudaStream_t stream
     CUresult cr = encode_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.X, (uint64_t)a.K, (uint64_t)a.M,
                                        (uint64_t)a.K * 2, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    cr = encode_tensor_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.qweight, (uint64_t)a.K * BITS / 32,
-                              (uint64_t)a.N, (uint64_t)a.K * BITS / 8, kWordsPerRowStage, kBN,
-                              BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B);
+    if constexpr (BITS == 16)
+        cr = encode_tensor_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.qweight, (uint64_t)a.K, (uint64_t)a.N,
+                                  (uint64_t)a.K * 2, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        cr = encode_tensor_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.qweight, (uint64_t)a.K * BITS / 32,
+                                  (uint64_t)a.N, (uint64_t)a.K * BITS / 8, kWordsPerRowStage, kBN,
+                                  BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B);
     if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
     cudaLaunchConfig_t cfg = {};
@@ -364,12 +378,15 @@ cudaError_t launch_gemm_bits(const GemmArgs& a, int num_sms, cudaStream_t stream
 
 static_assert(GemmSmem<2, 4>::kAlloc <= 227 * 1024, "4-bit GEMM shared memory");
 static_assert(GemmSmem<2, 8>::kAlloc <= 227 * 1024, "8-bit GEMM shared memory");
+static_assert(GemmSmem<2, 16>::kAlloc <= 227 * 1024, "bf16 GEMM shared memory");
+static_assert(GemmSmem<1, 16>::kAlloc <= 227 * 1024, "bf16 GEMM shared memory");
 
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, const LaunchOptions& opt, cudaStream_t stream) {
     (void)opt;
     if (a.bits == 8) return launch_gemm_bits<8>(a, num_sms, stream);
+    if (a.bits == 16) return launch_gemm_bits<16>(a, num_sms, stream);
     return launch_gemm_bits<4>(a, num_sms, stream);
 }
 

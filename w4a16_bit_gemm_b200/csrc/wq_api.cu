@@ -10,7 +10,6 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include <cublas_v2.h>
 #include <mutex>
 
 #include "../../include/wq.h"
@@ -308,9 +307,6 @@ AwqWorkspace awq_workspace(int64_t N, int64_t K, int64_t T, int64_t g) {
     return w;
 }
 
-std::mutex g_blas_mu;
-cublasHandle_t g_blas[kMaxDevices] = {};
-
 }  // namespace
 
 size_t wq_awq_workspace_bytes(int64_t d_out, int64_t d_in, int64_t T, int32_t group_size) {
@@ -348,21 +344,24 @@ wq_status wq_awq_search(const void* W_bf16, int64_t d_out, int64_t d_in, const v
     const uint16_t* W = static_cast<const uint16_t*>(W_bf16);
     const uint16_t* X = static_cast<const uint16_t*>(X_bf16);
 
-    // reference output Y = X W^T (fp32 accumulation), a plain library GEMM; the
-    // per-device handle is shared, so its stream is set and the GEMM enqueued
-    // under one lock
-    {
-        std::lock_guard<std::mutex> lk(g_blas_mu);
-        if (!g_blas[st.dev] && cublasCreate(&g_blas[st.dev]) != CUBLAS_STATUS_SUCCESS) return WQ_ERR_CUDA;
-        cublasHandle_t h = g_blas[st.dev];
-        const float one = 1.0f, zero = 0.0f;
-        if (cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS ||
-            cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, (int)d_out, (int)T, (int)d_in, &one, W, CUDA_R_16BF,
-                         (int)d_in, X, CUDA_R_16BF, (int)d_in, &zero, Yref, CUDA_R_32F, (int)d_out,
-                         CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-            return WQ_ERR_CUDA;
-    }
-    cudaError_t e = launch_awq_colstats(X, T, d_in, lnm, mean_ln, s);
+    // reference output Y = X W^T on the unquantized weights (fp32 accumulation):
+    // the tcgen05 GEMM with bf16 B tiles loaded by TMA
+    GemmArgs ga = {};
+    ga.X = X;
+    ga.qweight = reinterpret_cast<const uint32_t*>(W);
+    ga.Y = Yref;
+    ga.status = st.status;
+    ga.M = (int)T;
+    ga.N = (int)d_out;
+    ga.K = (int)d_in;
+    ga.g = (int)d_in;
+    ga.G = 1;
+    ga.y_fp32 = 1;
+    ga.bits = 16;
+    LaunchOptions gopt;
+    gopt.pdl = false;
+    cudaError_t e = launch_gemm(ga, st.num_sms, gopt, s);
+    if (e == cudaSuccess) e = launch_awq_colstats(X, T, d_in, lnm, mean_ln, s);
     for (int i = 0; e == cudaSuccess && i < kAwqAlphas; ++i) {
         e = launch_awq_scale_apply(W, d_out, X, T, d_in, lnm, mean_ln, i, nullptr, sbuf, Wp, Xp, st.num_sms, s);
         if (e == cudaSuccess)

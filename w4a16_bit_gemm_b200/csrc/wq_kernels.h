@@ -96,7 +96,8 @@ struct GemmArgs {
     int M, N, K, G, g;
     int symmetric;
     int y_fp32;
-    int bits;  // 4 (qweight [N][K/8], nibbles) or 8 (qweight [N][K/4], symmetric bytes)
+    int bits;  // 4 (qweight [N][K/8], nibbles), 8 (qweight [N][K/4], symmetric bytes) or
+               // 16 (qweight: unquantized bf16 [N][K]; scales, zeros unused)
 };
 
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, const LaunchOptions& opt, cudaStream_t stream);
