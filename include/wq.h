@@ -96,6 +96,18 @@ typedef enum {
 /* ABI version of the loaded library (WQ_ABI_VERSION). */
 int32_t wq_abi_version(void);
 
+/*
+ * Host-side fault injection, for testing a caller's error handling without a
+ * GPU fault (the pages' monitoring section: failures surfaced and alerted).
+ * With WQ_FAULT_INJECT=launch or WQ_FAULT_INJECT=alloc in the environment
+ * (read once per process), every entry point that would enqueue work fails
+ * after its argument checks: "alloc" at the per-device set-up that reserves
+ * device memory, "launch" at the last host step before the launch.  The call
+ * returns WQ_ERR_CUDA with nothing enqueued and the context untouched.
+ * wq_fault_injections returns how many calls failed that way in this process.
+ */
+uint64_t wq_fault_injections(void);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* wq_status_string(wq_status status);
 

@@ -176,3 +176,89 @@ def test_awq_static_rejects_before_any_device_work(lib):
     st = lib.wq_awq_search_static(FAKE, 8192, 8192, FAKE, 512, 128, 0, FAKE, FAKE, FAKE, FAKE, None, None, None)
     assert st == 2
     assert lib.wq_awq_search_static(None, 64, 256, FAKE, 8, 128, 0, FAKE, FAKE, FAKE, FAKE, None, None, None) == 1
+
+
+# ---------------------------------------------------------------------------
+# Host-side fault injection (WQ_FAULT_INJECT=launch|alloc): every entry point
+# that enqueues work fails with WQ_ERR_CUDA after its argument checks and
+# before any CUDA call, and each such failure is counted.  Runs in a child
+# process per mode (the variable is read once per process).
+# ---------------------------------------------------------------------------
+
+_INJECT_SCRIPT = r'''
+import ctypes, json, sys
+sys.path.insert(0, sys.argv[1])
+from w4a16_bit_gemm_b200 import binding
+lib = binding.lib
+F = 0x10000
+out = {}
+def call(name, *args):
+    before = lib.wq_fault_injections()
+    st = getattr(lib, name)(*args)
+    out[name] = [st, lib.wq_fault_injections() - before]
+call("wq_quantize_rtn", F, 4, 256, 128, 0, F, F, F, None)
+call("wq_quantize_clip_mse", F, 4, 256, 128, 0, F, F, F, None)
+call("wq_dequantize", F, F, F, 4, 256, 128, 0, F, None)
+call("wq_linear_w4a16", F, 1, F, F, F, 64, 256, 128, 0, F, 0, None, 0, None)
+call("wq_linear_w4a16", F, 300, F, F, F, 64, 256, 128, 0, F, 1, None, 0, None)
+ws = lib.wq_awq_workspace_bytes(64, 256, 8, 128)
+call("wq_awq_search", F, 64, 256, F, 8, 128, 0, F, F, F, F, None, None, F, ws, None)
+call("wq_awq_search_static", F, 64, 256, F, 8, 128, 0, F, F, F, F, None, None, None)
+call("wq_awq_scale_activations", F, 8, 256, F, F, None)
+call("wq_quantize_w8", F, 4, 256, 128, F, F, None)
+call("wq_dequantize_w8", F, F, 4, 256, 128, F, None)
+call("wq_linear_w8a16", F, 1, F, F, 64, 256, 128, F, 0, None)
+gws = lib.wq_gptq_workspace_bytes(64, 256)
+call("wq_gptq", F, 64, 256, F, 8, 128, 1, 1, F, F, None, None, F, gws, None)
+call("wq_get_device_error", None, None)
+call("wq_selftest_bounded_wait", 1000, None)
+# argument errors are still reported as such, with nothing counted
+
+before = lib.wq_fault_injections()
+out["invalid"] = [lib.wq_quantize_rtn(None, 4, 256, 128, 0, F, F, F, None), lib.wq_fault_injections() - before]
+print(json.dumps(out))
+'''
+
+ENQUEUEING = ["wq_quantize_rtn", "wq_quantize_clip_mse", "wq_dequantize", "wq_linear_w4a16", "wq_awq_search",
+              "wq_awq_search_static", "wq_awq_scale_activations", "wq_quantize_w8", "wq_dequantize_w8",
+              "wq_linear_w8a16", "wq_gptq", "wq_get_device_error", "wq_selftest_bounded_wait"]
+
+
+def _run_injected(mode):
+    import json
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    env.pop("WQ_FAULT_INJECT", None)
+    if mode:
+        env["WQ_FAULT_INJECT"] = mode
+    env["CUDA_VISIBLE_DEVICES"] = ""  # never reach a device, even on a GPU box
+    r = subprocess.run([sys.executable, "-c", _INJECT_SCRIPT, ROOT], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    return json.loads(r.stdout.strip().splitlines()[-1])
+
+
+def test_fault_injection_covers_every_enqueueing_entry_point(lib):
+    declared = set(declared_functions())
+    assert set(ENQUEUEING) <= declared
+    # the others only compute sizes or strings and never enqueue work
+    assert declared - set(ENQUEUEING) == {"wq_abi_version", "wq_status_string", "wq_linear_workspace_bytes",
+                                          "wq_awq_workspace_bytes", "wq_awq_static_scratch_bytes",
+                                          "wq_gptq_workspace_bytes", "wq_fault_injections"}
+
+
+@pytest.mark.parametrize("mode", ["launch", "alloc"])
+def test_fault_injection_fails_each_call_once(lib, mode):
+    out = _run_injected(mode)
+    for name in ENQUEUEING:
+        st, counted = out[name]
+        assert st == 3 and counted == 1, (mode, name, st, counted)  # WQ_ERR_CUDA, one injected failure
+    assert out["invalid"] == [1, 0]  # WQ_ERR_INVALID_ARG first, nothing injected
+
+
+def test_no_injection_without_the_variable(lib):
+    out = _run_injected(None)
+    for name in ENQUEUEING:
+        assert out[name][1] == 0, name
+    assert out["invalid"] == [1, 0]

@@ -181,3 +181,33 @@ def test_gemv_m1_large_rows_fallback():
     X = bf16_bits_of(rng.standard_normal((1, K)))
     cols = np.sort(rng.choice(N, 300, replace=False))
     run_case(W, X, 128, False, torch.float32, cols=cols)
+
+
+def test_injected_launch_failure_leaves_outputs_untouched():
+    """WQ_FAULT_INJECT=launch in a child process on the GPU: the linear layer
+    returns WQ_ERR_CUDA, its output buffer keeps the caller's sentinel and the
+    device status stays clean (nothing was enqueued)."""
+    import os
+    import subprocess
+    import sys
+    script = r'''
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+from w4a16_bit_gemm_b200 import binding as b
+W = torch.randn(256, 512, device="cuda").to(torch.bfloat16)
+q = torch.zeros(256, 64, dtype=torch.int32, device="cuda")
+s = torch.ones(256, 4, dtype=torch.float16, device="cuda")
+z = torch.zeros(256, 4, dtype=torch.float16, device="cuda")
+X = torch.randn(1, 512, device="cuda").to(torch.bfloat16)
+Y = torch.full((1, 256), 7.0, device="cuda")
+st = b.lib.wq_linear_w4a16(X.data_ptr(), 1, q.data_ptr(), s.data_ptr(), z.data_ptr(), 256, 512, 128, 0,
+                           Y.data_ptr(), 1, None, 0, torch.cuda.current_stream().cuda_stream)
+torch.cuda.synchronize()
+print(st, int(b.lib.wq_fault_injections()), bool(torch.all(Y == 7.0)))
+'''
+    env = dict(os.environ, WQ_FAULT_INJECT="launch")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", script, root], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    st, n, untouched = r.stdout.split()[-3:]
+    assert st == "3" and n == "1" and untouched == "True"

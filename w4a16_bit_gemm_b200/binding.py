@@ -82,6 +82,8 @@ def _load() -> ctypes.CDLL:
     lib.wq_get_device_error.restype = ctypes.c_int
     lib.wq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     lib.wq_selftest_bounded_wait.restype = ctypes.c_int
+    lib.wq_fault_injections.argtypes = []
+    lib.wq_fault_injections.restype = ctypes.c_uint64
     return lib
 
 

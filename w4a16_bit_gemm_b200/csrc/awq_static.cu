@@ -32,6 +32,9 @@ extern "C" wq_status wq_awq_search_static(const void* W_bf16, int64_t d_out, int
                                      zeros_fp16, s_bf16, losses, best);
     if (v != WQ_OK) return v;
     if (wq_awq_workspace_bytes(d_out, d_in, T, group_size) > kAwqStaticScratchBytes) return WQ_ERR_UNSUPPORTED;
+    // the scratch's set-up (symbol lookup) comes before the search's own: both
+    // injected faults land here
+    if (wq::fault_injected(wq::kFaultAlloc) || wq::fault_injected(wq::kFaultLaunch)) return WQ_ERR_CUDA;
     void* ws = nullptr;
     if (cudaGetSymbolAddress(&ws, g_awq_static_scratch) != cudaSuccess) return WQ_ERR_CUDA;
     return wq_awq_search(W_bf16, d_out, d_in, X_bf16, T, group_size, symmetric, qweight, scales_fp16, zeros_fp16,

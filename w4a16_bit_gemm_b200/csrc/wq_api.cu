@@ -10,6 +10,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/wq.h"
@@ -19,6 +20,27 @@ namespace wq {
 
 // Device status word (WQ_DEVFLAG_* bits), one per device that loads the library.
 __device__ uint32_t g_status_word;
+
+// Host-side fault injection (WQ_FAULT_INJECT=launch|alloc, read once per
+// process): the named step fails as a CUDA error would, before anything is
+// enqueued, and the call returns WQ_ERR_CUDA; every such failure is counted.
+namespace {
+std::atomic<uint64_t> g_fault_count{0};
+int fault_mode() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("WQ_FAULT_INJECT");
+        v = !e ? kFaultNone : strcmp(e, "launch") == 0 ? kFaultLaunch : strcmp(e, "alloc") == 0 ? kFaultAlloc : kFaultNone;
+    }
+    return v;
+}
+}  // namespace
+
+bool fault_injected(int step) {
+    if (fault_mode() != step) return false;
+    g_fault_count.fetch_add(1);
+    return true;
+}
 
 namespace {
 
@@ -43,6 +65,9 @@ struct DeviceState {
 // Per-device set-up on first use: address of the status word, SM count.
 // Must not run inside a stream capture (it may load the module).
 wq_status device_state(DeviceState* st) {
+    // the per-device set-up reserves device memory (module load) and is the
+    // last host step before every launch: both injected faults land here
+    if (fault_injected(kFaultAlloc) || fault_injected(kFaultLaunch)) return WQ_ERR_CUDA;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WQ_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
@@ -149,6 +174,8 @@ using namespace wq;
 extern "C" {
 
 int32_t wq_abi_version(void) { return WQ_ABI_VERSION; }
+
+uint64_t wq_fault_injections(void) { return g_fault_count.load(); }
 
 const char* wq_status_string(wq_status s) {
     switch (s) {

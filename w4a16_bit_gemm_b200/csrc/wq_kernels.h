@@ -9,6 +9,11 @@
 
 namespace wq {
 
+// Host-side fault injection (WQ_FAULT_INJECT): true when the named step is to
+// fail in this process (the failure is counted for wq_fault_injections).
+enum FaultStep { kFaultNone = 0, kFaultLaunch = 1, kFaultAlloc = 2 };
+bool fault_injected(int step);
+
 cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric, uint32_t* qweight,
                             uint16_t* scales, uint16_t* zeros, uint32_t* status, int num_sms, cudaStream_t stream);
 
