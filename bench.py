@@ -254,6 +254,52 @@ def bench_gemv_shape(b, syn, wl, ci, M, copies, steps, warmup, dist):
             "GBps": nbytes / per_launch / 1e9, "bytes_per_launch": nbytes}
 
 
+def bench_whole_model(b, syn, args, dist, hbm):
+    """Config 5: quantize the 160 weight matrices of a 32-layer 7B-shaped
+    decoder (qkv, o, gate, up, down), report the artifact bytes against
+    P*4/8 + scale/zero bytes, then time one M=1 decode sweep over the 160
+    layers in model order (one CUDA graph; 3.44 GB of artifacts per sweep, far
+    above L2, so every launch streams from HBM)."""
+    wl = syn.WHOLE_MODEL
+    cases = wl.cases
+    Ws = [syn.case_weight(wl, i, "cuda") for i in range(len(cases))]
+    packs = [b.quantize_rtn(W, 128, False) for W in Ws]  # allocation + warm-up
+    torch.cuda.synchronize()
+    P = sum(c.d_out * c.d_in for c in cases)
+    art = sum(p.nbytes() for p in packs)
+    qbytes = sum(quant_bytes(c.d_out, c.d_in, False) for c in cases)
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    e0.record()
+    for _ in range(reps):
+        for W, p in zip(Ws, packs):
+            b.quantize_rtn(W, 128, False, out=p)
+    e1.record()
+    torch.cuda.synchronize()
+    tq = dist.max(e0.elapsed_time(e1) / 1e3) / reps
+    del Ws
+    torch.cuda.empty_cache()
+    X = [syn.case_activations(wl, i, 1, "cuda") for i in range(len(cases))]
+    Y = [torch.empty(1, c.d_out, dtype=torch.bfloat16, device="cuda") for c in cases]
+
+    def sweep():
+        for i, p in enumerate(packs):
+            b.linear_w4a16(X[i], p, out=Y[i])
+    g = capture(sweep)
+    steps = max(10, min(200, args.steps))
+    t = dist.max(timed_graph(g, steps, 3, dist)) / steps
+    sweep_bytes = sum(gemv_bytes(c.d_out, c.d_in, 1, False) for c in cases)
+    del g, packs, X, Y
+    torch.cuda.empty_cache()
+    return {"layers": len(cases), "params": P, "artifact_bytes": art,
+            "payload_bytes_P_x_4_over_8": P * 4 // 8, "scale_zero_bytes": art - P * 4 // 8,
+            "bits_per_weight": 8.0 * art / P,
+            "quantize_all_ms": tq * 1e3, "quantize_all_GBps": qbytes / tq / 1e9,
+            "gemv_sweep_ms": t * 1e3, "gemv_sweep_bytes": sweep_bytes, "gemv_sweep_GBps": sweep_bytes / t / 1e9,
+            "gemv_sweep_frac_of_measured_hbm": sweep_bytes / t / 1e9 / hbm}
+
+
 def run_ours(args, dist: Dist):
     from w4a16_bit_gemm_b200 import binding as b
     from w4a16_bit_gemm_b200 import synthetic as syn
@@ -494,7 +540,7 @@ def run_ours(args, dist: Dist):
         Xg = syn.case_activations(syn.PREFILL, ci, M, "cuda")
         Yg = torch.empty(M, cc.d_out, dtype=torch.bfloat16, device="cuda")
         gg = capture(lambda: b.linear_w4a16(Xg, pg, out=Yg))
-        gsteps = max(3, min(50, args.steps // 40))
+        gsteps = max(20, min(50, args.steps // 40))
         tg = dist.max(timed_graph(gg, gsteps, 2, dist)) / gsteps
         flops = 2.0 * M * cc.d_out * cc.d_in
         tfl = flops / tg / 1e12
@@ -503,10 +549,24 @@ def run_ours(args, dist: Dist):
                                   "frac_of_measured_bf16_sustained": tfl / tf_sust})
         del gg, pg, Xg, Yg
         torch.cuda.empty_cache()
+    # ---------------- config 5: the whole 7B-shaped decoder weight set ----------------
+    secondary["whole_model"] = bench_whole_model(b, syn, args, dist, hbm)
+
     clocks = sampler.stop()
     st, flags = b.device_error()
     if st != b.WQ_OK:
         raise RuntimeError(f"device status after the bench: {st} flags {flags}")
+
+    # the numbers the metric names, last on the line (a stored tail keeps them)
+    g_by = {(r["shape"], r["M"]): r for r in secondary["gemv"]}
+    secondary["summary"] = {
+        "quantize_GBps": secondary["quantize"]["GBps"],
+        "dequantize_GBps": secondary["dequantize"]["GBps"],
+        "gemm_TFLOPs": {f"{r['M']}x{r['N']}x{r['K']}": r["TFLOPs"] for r in secondary["gemm"]},
+        "gemv_GBps": {f"{k[0]} M={k[1]}": v["GBps"] for k, v in g_by.items()},
+        "whole_model": {k: secondary["whole_model"][k] for k in ("quantize_all_GBps", "artifact_bytes",
+                                                                  "gemv_sweep_GBps", "gemv_sweep_frac_of_measured_hbm")},
+    }
 
     traffic = kernel_traffic("gemv_traffic.json")
 
@@ -561,6 +621,27 @@ def oracle_gemv_sample(n_launch: int, nthreads: int | None = None):
         oracle.linear(Xb, W_hat, nthreads)
     dt = time.perf_counter() - t0
     return gemv_bytes(D, D, 1, False) * n_launch / dt / 1e9, nthreads, dt
+
+
+def oracle_quant_sample(nthreads: int | None = None, reps: int = 1):
+    """The oracle's quantize+pack and dequantize of the 4096x4096 attention
+    projection (bf16 in, packed codes / bf16 out), as GB/s of the same
+    algorithmic bytes the GPU numbers use."""
+    import oracle
+    from w4a16_bit_gemm_b200 import synthetic as syn
+    W = syn.case_weight(syn.ATTN, 0, "cpu")
+    Wb = W.view(torch.int16).numpy().view(np.uint16)
+    nthreads = nthreads or oracle.default_threads()
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        q, s, z, _, codes = oracle.quantize_pack4(Wb, 128, False, nthreads=nthreads)
+    tq = (time.perf_counter() - t0) / reps
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.dequantize(codes, s, z, 128, nthreads)
+    td = (time.perf_counter() - t0) / reps
+    qb = quant_bytes(D, D, False)
+    return qb / tq / 1e9, qb / td / 1e9, nthreads
 
 
 def calibrated_sample(target_s: float = 12.0):
@@ -619,11 +700,17 @@ def main():
             if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
                 v, n, dt, nl = calibrated_sample()
                 v1, _, dt1 = oracle_gemv_sample(2, nthreads=1)
+                qv, dv, _ = oracle_quant_sample(reps=2)
+                qv1, dv1, _ = oracle_quant_sample(nthreads=1)
                 out["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": n, "kind": "oracle",
                                        "sample": f"{nl} GEMV launch(es) of the 4096x4096 M=1 workload "
                                                  f"(unpack + dequantize + fp64 linear), {dt:.1f} s",
                                        "single_thread_value": v1,
-                                       "single_thread_sample": f"2 launches on 1 core, {dt1:.1f} s"}
+                                       "single_thread_sample": f"2 launches on 1 core, {dt1:.1f} s",
+                                       "quantize_GBps": qv, "dequantize_GBps": dv,
+                                       "quantize_GBps_1_core": qv1, "dequantize_GBps_1_core": dv1,
+                                       "quantize_sample": "quantize+pack and dequantize of W[4096,4096] g128 asym, "
+                                                          f"2 reps on {n} cores, 1 rep on 1 core"}
         if out is not None and dist.rank == 0:
             print(json.dumps(out), flush=True)
     finally:
