@@ -171,48 +171,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool nvalid = n < a.N;
         const bool sym = a.symmetric != 0;
         const int kw = a.K * BITS / 32;  // packed words per row
-        // Scale (and zero) of the two 32-k halves of k block kb, packed as
-        // (scale | zero << 16), loaded kPre k blocks ahead of their use so that
-        // no k block waits on a global load.
-        constexpr int kPre = 4;
-        uint32_t szA[kPre], szB[kPre];
-        auto load_sz = [&](int kb, uint32_t& za, uint32_t& zb) {
-            za = zb = 0x3c00u;  // s = 1, z = 0 past the row's end (or past K)
-            const int kbase = kb * kBK;
-            if (!nvalid || kbase >= a.K) return;
-            const int gA = kbase / a.g, gB = (kbase + 32) / a.g;
-            const int64_t ia = (int64_t)n * a.G + gA;
-            za = (uint32_t)ld_nc_u16(a.scales + ia) | (sym ? 0u : (uint32_t)ld_nc_u16(a.zeros + ia) << 16);
-            zb = za;
-            if (gB != gA && kbase + 32 < a.K) {
-                const int64_t ib = (int64_t)n * a.G + gB;
-                zb = (uint32_t)ld_nc_u16(a.scales + ib) | (sym ? 0u : (uint32_t)ld_nc_u16(a.zeros + ib) << 16);
-            }
-        };
-#pragma unroll
-        for (int p = 0; p < kPre; ++p) load_sz(p, szA[p], szB[p]);
         for (int kb = 0; kb < (BITS == 16 ? 0 : nkb); ++kb) {
             const int s1 = kb % kS1, s2 = kb % kS2;
             if (__any_sync(0xffffffffu, *(volatile int*)abort_flag != 0)) break;
-            // group constants for the two 32-k halves of this k block (loaded
-            // kPre blocks ago), then the load for block kb + kPre into the slot
+            // group constants for the two 32-k halves of this k block
             const int kbase = kb * kBK;
-            uint32_t za = 0, zb = 0;
-#pragma unroll
-            for (int p = 0; p < kPre; ++p)
-                if ((kb % kPre) == p) {
-                    za = szA[p];
-                    zb = szB[p];
-                    load_sz(kb + kPre, szA[p], szB[p]);
-                }
             const int gA = kbase / a.g, gB = (kbase + 32) / a.g;
             uint8_t* brow = smem + SL::kOffB + s2 * SL::kBTile + i * 128;
             if constexpr (BITS == 16) {
                 // no producer work: TMA loads the bf16 B tiles
             } else if constexpr (BITS == 4) {
-                const auto zf = [](uint32_t v) { return (int)__half2float(__ushort_as_half((uint16_t)(v >> 16))); };
-                const GroupConsts cA = make_group_consts((uint16_t)(za & 0xffffu), sym ? 0 : zf(za), sym);
-                const GroupConsts cB = make_group_consts((uint16_t)(zb & 0xffffu), sym ? 0 : zf(zb), sym);
+                GroupConsts cA, cB;
+                if (nvalid) {
+                    const int64_t ia = (int64_t)n * a.G + gA;
+                    cA = make_group_consts(a.scales[ia], sym ? 0 : (int)__half2float(__ushort_as_half(a.zeros[ia])), sym);
+                    if (gB != gA && kbase + 32 < a.K) {
+                        const int64_t ib = (int64_t)n * a.G + gB;
+                        cB = make_group_consts(a.scales[ib], sym ? 0 : (int)__half2float(__ushort_as_half(a.zeros[ib])),
+                                               sym);
+                    } else {
+                        cB = cA;
+                    }
+                } else {
+                    cA = make_group_consts(0x3c00u, 0, sym);
+                    cB = cA;
+                }
                 bool ready = mbar_wait(&full1[s1], (uint32_t)(kb / kS1) & 1u, a.status);
                 if (ready && kb >= kS2) ready = mbar_wait(&empty2[s2], (uint32_t)((kb / kS2) - 1) & 1u, a.status);
                 if (!__all_sync(0xffffffffu, ready)) {  // warp-uniform give-up
@@ -240,11 +223,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     *reinterpret_cast<uint4*>(brow + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
                 }
             } else {
-                // symmetric INT8: scales only (zero scales past the row's end)
-                const float sA = nvalid ? __half2float(__ushort_as_half((uint16_t)(za & 0xffffu))) : 0.0f;
-                const float sB = nvalid ? __half2float(__ushort_as_half((uint16_t)(zb & 0xffffu))) : 0.0f;
-                (void)gA;
-                (void)gB;
+                float sA = 0.0f, sB = 0.0f;  // symmetric INT8: scales only
+                if (nvalid) {
+                    sA = __half2float(__ushort_as_half(a.scales[(int64_t)n * a.G + gA]));
+                    sB = (gB != gA && kbase + 32 < a.K) ? __half2float(__ushort_as_half(a.scales[(int64_t)n * a.G + gB]))
+                                                         : sA;
+                }
                 bool ready = mbar_wait(&full1[s1], (uint32_t)(kb / kS1) & 1u, a.status);
                 if (ready && kb >= kS2) ready = mbar_wait(&empty2[s2], (uint32_t)((kb / kS2) - 1) & 1u, a.status);
                 if (!__all_sync(0xffffffffu, ready)) {  // warp-uniform give-up
