@@ -9,12 +9,12 @@
 //
 // Data layout: the weights are a flat row-major array, so group gi covers the
 // elements [gi*g, (gi+1)*g) and its scale/zero live at index gi; packed word w
-// holds elements [8w, 8w+8).  A "segment" is 8 consecutive weights = one
-// 16-byte load and one packed output word.  For g <= 256 one group spans
-// L = g/8 lanes of a warp; the min/max is a butterfly shuffle over those
-// lanes.  For larger g one warp owns a group and loops over it twice.
-// All loads/stores are 128-bit (input) and 32-bit (packed output), fully
-// coalesced: consecutive lanes touch consecutive addresses.
+// holds elements [8w, 8w+8).  For g <= 256 (quantize_stream_kernel) a copy
+// warp streams 32-weight units into shared memory with TMA, one consumer
+// thread quantizes one unit, and a group spans L = g/32 lanes (butterfly
+// shuffles for its min/max).  For larger g (quantize_large_group_kernel) one
+// warp owns a group and loops over it twice.  Outputs are written with
+// coalesced stores: consecutive lanes touch consecutive addresses.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -68,54 +68,6 @@ __device__ __forceinline__ ScaleZero scale_zero(float lo, float hi, bool symmetr
         float zf = rintf(__fsub_rn(0.0f, __fdiv_rn(lo, s)));
         zf = fminf(fmaxf(zf, 0.0f), 15.0f);
         r.z = (int)zf;
-    }
-    return r;
-}
-
-// rcp.approx.f32: at most 1 ulp from 1/s.
-__device__ __forceinline__ float rcp_approx(float s) {
-    float r;
-    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(s));
-    return r;
-}
-
-// rint(fl32(-lo / s)) with the IEEE division (rare: near a half-integer).
-__device__ __noinline__ float exact_neg_quotient_rint(float lo, float s) {
-    return rintf(__fsub_rn(0.0f, __fdiv_rn(lo, s)));
-}
-
-// scale_zero without fp32 divisions on the common path.
-//  - fl32(r / 15) (or / 7) equals fl32(fl64(r) * fl64(1/15)): r has 24
-//    significant bits, so a quotient that is not exact lies at least 2^-29
-//    (relative) away from every fp32 rounding midpoint, while the fp64
-//    product is within 2^-52 of the quotient (correct rounding of the
-//    quotient is preserved).
-//  - z = rint(fl32(-lo / s)) through f = -lo * rcp(s) with the quotient
-//    guard of rint_quotient (the exact division decides near a half-integer).
-// Also returns rcp(s) for the code path.
-__device__ __forceinline__ ScaleZero scale_zero_fast(float lo, float hi, bool symmetric, float& rcp_out) {
-    float s32;
-    if (symmetric)
-        s32 = __double2float_rn((double)fmaxf(-lo, hi) * (1.0 / 7.0));
-    else
-        s32 = __double2float_rn((double)__fsub_rn(hi, lo) * (1.0 / 15.0));
-    ScaleZero r;
-    r.s16 = __half_as_ushort(__float2half_rn(s32));
-    r.range = false;
-    r.z = 0;
-    if (r.s16 == 0x7c00u) {  // fp16 overflow: saturate
-        r.s16 = 0x7bffu;
-        r.range = true;
-    }
-    if (r.s16 == 0u) r.s16 = 0x3c00u;  // all-zero or underflowing group
-    const float s = __half2float(__ushort_as_half(r.s16));
-    const float rcp = rcp_approx(s);
-    rcp_out = rcp;
-    if (!symmetric && lo != 0.0f) {
-        const float f = __fmul_rn(-lo, rcp);
-        float t = rintf(f);
-        if (fabsf(f) < 32.0f && fabsf(__fsub_rn(f, t)) > 0.5f - 0x1p-17f) t = exact_neg_quotient_rint(lo, s);
-        r.z = (int)fminf(fmaxf(t, 0.0f), 15.0f);
     }
     return r;
 }
@@ -178,157 +130,247 @@ __device__ __noinline__ float2 nan_skipping_min_max(const uint4 r0, const uint4 
     return make_float2(lo, hi);
 }
 
-// Offset codes (q + z, or q + 8 when symmetric) of 16 packed bf16 pairs through
-// f = x * rcp and the rounding constant; dmax collects |f - rint(f)|.
-template <bool CLAMP>
-__device__ __forceinline__ void fast_codes(const uint32_t (&w)[16], float rcp, uint32_t coff, bool sym,
-                                           uint32_t (&word)[4], float& dmax) {
-    const float2 rcp2 = make_float2(rcp, rcp);
-    const float2 mag2 = make_float2(kRoundMagic, kRoundMagic);
-    const float2 nmag2 = make_float2(-kRoundMagic, -kRoundMagic);
-    const float2 neg1 = make_float2(-1.0f, -1.0f);
-    float dm0 = 0.0f, dm1 = 0.0f;
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        uint32_t acc = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t wv = w[4 * h + i];
-            const float2 x2 = make_float2(__uint_as_float(wv << 16), __uint_as_float(wv & 0xffff0000u));
-            const float2 f2 = __fmul2_rn(x2, rcp2);
-            const float2 t2 = __fadd2_rn(f2, mag2);
-            const float2 r2 = __fadd2_rn(t2, nmag2);    // rint(f), exact
-            const float2 d2 = __ffma2_rn(r2, neg1, f2);  // f - rint(f), exact
-            dm0 = fmaxf(dm0, fabsf(d2.x));
-            dm1 = fmaxf(dm1, fabsf(d2.y));
-            int c0 = (int)(__float_as_uint(t2.x) + coff), c1 = (int)(__float_as_uint(t2.y) + coff);
-            if (CLAMP) {  // offset codes: [0, 15] for both encodings
-                c0 = min(max(c0, 0), 15);
-                c1 = min(max(c1, 0), 15);
-            }
-            // elements 2i and 2i + 1 of the word: nibbles 2i and 2i + 1 (low first)
-            acc |= (uint32_t)c0 << (8 * i);
-            acc |= (uint32_t)c1 << (8 * i + 4);
-        }
-        word[h] = sym ? acc ^ 0x88888888u : acc;  // q + 8 -> two's-complement nibble
-    }
-    dmax = fmaxf(dm0, dm1);
-}
-
 __device__ __noinline__ uint32_t encode8_slow(const uint4 raw, const ScaleZero sz, bool symmetric) {
     float v[8];
     unpack_bf16x8(raw, v);
     return encode8(v, sz, symmetric);
 }
 
-// g <= 256: each thread takes four consecutive segments (32 weights, four
-// 16-byte loads), so the per-group work is shared by 32 weights per thread;
-// L = g/32 lanes per group, 32/L groups per warp.
+// ------------------------------------------------------------------------
+// Streaming quantize for g <= 256 (the common group sizes).
 //
-// Fast path (finite group, scale not saturated -- then |x/s| <= 15.01):
-//  - statistics with packed bf16x2 max/min that propagate NaN, so one test
-//    per thread tells whether its values are all non-NaN;
-//  - scale and zero without fp32 divisions (scale_zero_fast);
-//  - f = x * rcp(s) in packed fp32x2; t = f + 1.5*2^23 puts rint(f) (round
-//    half to even) in the low mantissa bits, so the code is bits(t) + const;
-//  - the quotient guard of rint_quotient: if some |f - rint(f)| is within
-//    2^-17 of 1/2, the thread redoes its codes with the IEEE division;
-//  - fl(x/s) and rint are monotone, so the codes of the group's extremes
-//    bound all its codes: when both are inside the code range (and neither
-//    is near a tie) no code needs clamping.
-// Anything else (NaN or Inf in the warp's groups, a saturated scale) takes
-// the general per-value path of encode8.
-constexpr int kUnitsPerThread = 2;  // 32-weight units in flight per thread
+// The weights are read as rows of one 32-weight unit (64 bytes): a copy warp
+// keeps a ring of kQsStages stages of 256 units (16 KB) in flight with 2D TMA
+// loads (SWIZZLE_64B, so the 64-byte rows read by consecutive threads fall on
+// different banks); each of the 256 consumer threads quantizes one unit per
+// stage.  Two CTAs per SM; the units are split evenly over the grid in whole
+// quanta of 8 units (whole groups for every g <= 256).
+//
+// Codes without a division and without a per-value test: with rcp = rn(1/s),
+// q0 = rn(x rcp), the residual r = fma(-q0, s, x) and q1 = fma(r, rcp, q0)
+// (Markstein's correction step for a correctly rounded reciprocal), q1 is the
+// IEEE quotient fl(x/s) wherever the quotient is not subnormal, and rint(q1)
+// equals rint(fl(x/s)) for every bf16 x and every finite fp16 s with
+// |x/s| <= 40 (checked exhaustively on the CPU over all such pairs).  Then
+// t = q1 + 1.5*2^23 puts rint(q1) (round half to even) in the low mantissa
+// bits and t + off adds the zero point (or 8) exactly.  fl(x/s) and rint are
+// monotone, so the codes of the group's extremes bound all its codes: when
+// both lie in [0, 15], no code needs clamping.
+// ------------------------------------------------------------------------
+constexpr int kQsWarps = 8;                         // consumer warps
+constexpr int kQsConsumers = kQsWarps * 32;         // one unit per thread per stage
+constexpr int kQsThreads = kQsConsumers + 32;       // + the copy warp
+constexpr int kQsStageBytes = kQsConsumers * 64;    // 16 KB
+constexpr int kQsStages = 4;
+constexpr int kQsCtasPerSm = 2;
+constexpr int kQsSmem = kQsStages * kQsStageBytes + 1024;  // + base alignment slack
+constexpr int64_t kQsMaxUnits = int64_t(1) << 30;   // units per launch (TMA coordinates are 32-bit)
 
-// Fast code of x (offset form: q + z, or q + 8 when symmetric) and |f - rint(f)|.
-__device__ __forceinline__ int fast_code(float x, float rcp, uint32_t coff, float& dist) {
-    const float f = __fmul_rn(x, rcp);
-    const float t = __fadd_rn(f, kRoundMagic);
-    dist = fabsf(__fsub_rn(f, __fsub_rn(t, kRoundMagic)));
-    return (int)(__float_as_uint(t) + coff);
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+    return r;
+}
+
+// fl(x/s) for two values through the corrected product (see above).
+__device__ __forceinline__ float2 quotient2(float2 x2, float2 rcp2, float2 ns2) {
+    const float2 q0 = __fmul2_rn(x2, rcp2);
+    const float2 r = __ffma2_rn(q0, ns2, x2);
+    return __ffma2_rn(r, rcp2, q0);
+}
+
+// Scale and zero exactly as scale_zero, with the zero point through the
+// corrected product; also returns rn(1/s).
+__device__ __forceinline__ ScaleZero scale_zero_rcp(float lo, float hi, bool symmetric, float& rcp) {
+    float s32;
+    if (symmetric)
+        s32 = __double2float_rn((double)fmaxf(-lo, hi) * (1.0 / 7.0));
+    else
+        s32 = __double2float_rn((double)__fsub_rn(hi, lo) * (1.0 / 15.0));
+    ScaleZero r;
+    r.s16 = __half_as_ushort(__float2half_rn(s32));
+    r.range = false;
+    r.z = 0;
+    if (r.s16 == 0x7c00u) {  // fp16 overflow: saturate
+        r.s16 = 0x7bffu;
+        r.range = true;
+    }
+    if (r.s16 == 0u) r.s16 = 0x3c00u;  // all-zero or underflowing group
+    const float s = __half2float(__ushort_as_half(r.s16));
+    rcp = __frcp_rn(s);
+    if (!symmetric && lo != 0.0f) {
+        if (isinf(lo)) {
+            r.z = 15;  // rint(-lo/s) = +inf, clamped
+        } else {
+            // -lo/s >= 0; a quotient far above 15 stays far above it
+            const float y = __fsub_rn(0.0f, lo);
+            const float q0 = __fmul_rn(y, rcp);
+            const float q1 = __fmaf_rn(__fmaf_rn(q0, -s, y), rcp, q0);
+            r.z = (int)fminf(rintf(q1), 15.0f);
+        }
+    }
+    return r;
+}
+
+// Offset codes (q + z, or q + 8 when symmetric, as nibbles low first) of 16
+// packed bf16 pairs.
+template <bool CLAMP>
+__device__ __forceinline__ void exact_codes(const uint32_t (&w)[16], float rcp, float s, float off, bool sym,
+                                            uint32_t (&word)[4]) {
+    const float2 rcp2 = make_float2(rcp, rcp), ns2 = make_float2(-s, -s);
+    const float2 m2 = make_float2(kRoundMagic, kRoundMagic), off2 = make_float2(off, off);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        uint32_t b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t wv = w[4 * h + i];
+            const float2 x2 = make_float2(__uint_as_float(wv << 16), __uint_as_float(wv & 0xffff0000u));
+            const float2 t = __fadd2_rn(__fadd2_rn(quotient2(x2, rcp2, ns2), m2), off2);
+            const uint32_t l0 = __float_as_uint(t.x), l1 = __float_as_uint(t.y);
+            if (CLAMP) {
+                const int c0 = min(max((int)(l0 - kRoundMagicBits), 0), 15);
+                const int c1 = min(max((int)(l1 - kRoundMagicBits), 0), 15);
+                b[i] = (uint32_t)c0 | ((uint32_t)c1 << 4);
+            } else {
+                b[i] = l1 * 16u + l0;  // low byte: (code1 << 4) | code0, both in [0, 15]
+            }
+        }
+        const uint32_t lo2 = __byte_perm(b[0], b[1], 0x0040), hi2 = __byte_perm(b[2], b[3], 0x0040);
+        const uint32_t acc = __byte_perm(lo2, hi2, 0x5410);
+        word[h] = sym ? acc ^ 0x88888888u : acc;  // q + 8 -> two's-complement nibble
+    }
 }
 
 template <int L>
-__global__ void __launch_bounds__(kQuantThreads) quantize_small_group_kernel(
-    const uint4* __restrict__ W, int64_t nunit, int symmetric, uint32_t* __restrict__ qweight,
+__global__ void __launch_bounds__(kQsThreads, kQsCtasPerSm) quantize_stream_kernel(
+    const __grid_constant__ CUtensorMap tmap, int64_t nunit, int symmetric, uint32_t* __restrict__ qweight,
     uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros, uint32_t* status) {
-    const int lane = threadIdx.x & 31;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* stages = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ uint64_t full[kQsStages], empty[kQsStages];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // the CTA's units [u0, u1): quanta of 8 units split evenly over the grid
+    const int64_t nq = (nunit + 7) / 8;
+    const int64_t per = nq / gridDim.x, extra = nq - per * gridDim.x;
+    const int64_t u0 = 8 * ((int64_t)blockIdx.x * per + min((int64_t)blockIdx.x, extra));
+    const int64_t u1 = min(u0 + 8 * (per + ((int64_t)blockIdx.x < extra ? 1 : 0)), nunit);
+    const int nst = u1 > u0 ? (int)((u1 - u0 + kQsConsumers - 1) / kQsConsumers) : 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kQsStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kQsWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kQsWarps) {
+        // ---------------- copy warp ----------------
+        if (lane == 0) {
+            prefetch_tmap(&tmap);
+            for (int k = 0; k < nst; ++k) {
+                const int slot = k % kQsStages;
+                if (k >= kQsStages && !mbar_wait(&empty[slot], (uint32_t)((k / kQsStages) - 1) & 1u, status)) break;
+                mbar_arrive_expect_tx(&full[slot], kQsStageBytes);
+                tma_load_2d(stages + slot * kQsStageBytes, &tmap, &full[slot], 0,
+                            (int32_t)(u0 + (int64_t)k * kQsConsumers));
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumers: one unit per thread per stage ----------------
     const bool sym = symmetric != 0;
     bool nonfinite = false, range = false;
-    const int64_t stride = (int64_t)gridDim.x * (kQuantThreads * kUnitsPerThread);
-    for (int64_t base = (int64_t)blockIdx.x * (kQuantThreads * kUnitsPerThread) + threadIdx.x;
-         base - threadIdx.x < nunit; base += stride) {
-        uint4 raw[kUnitsPerThread][4];
+    // row threadIdx.x of a stage; its 16-byte chunk c sits at c ^ ((row >> 1) & 3)
+    const uint32_t row_addr = smem_u32(stages) + threadIdx.x * 64;
+    const uint32_t swz = (threadIdx.x >> 1) & 3;
+    for (int k = 0; k < nst; ++k) {
+        const int slot = k % kQsStages;
+        const bool ok = mbar_wait(&full[slot], (uint32_t)(k / kQsStages) & 1u, status);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        uint4 raw[4];
+        const uint32_t a = row_addr + slot * kQsStageBytes;
 #pragma unroll
-        for (int u = 0; u < kUnitsPerThread; ++u) {
-            const int64_t un = base + (int64_t)u * kQuantThreads;
+        for (int v = 0; v < 4; ++v) raw[v] = ld_shared_u4(a + (((uint32_t)v ^ swz) << 4));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+
+        const int64_t un = u0 + (int64_t)k * kQsConsumers + threadIdx.x;
+        const bool valid = un < u1;
+        uint32_t w[16];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) raw[u][v] = un < nunit ? ld_nc_v4(W + 4 * un + v) : make_uint4(0, 0, 0, 0);
+        for (int v = 0; v < 4; ++v) {
+            w[4 * v] = raw[v].x;
+            w[4 * v + 1] = raw[v].y;
+            w[4 * v + 2] = raw[v].z;
+            w[4 * v + 3] = raw[v].w;
+        }
+        // ---- statistics of the thread's 32 values (NaN propagates), as a tree ----
+        __nv_bfloat162 mx[8], mn[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            mx[i] = __hmax2_nan(bits_bf2(w[2 * i]), bits_bf2(w[2 * i + 1]));
+            mn[i] = __hmin2_nan(bits_bf2(w[2 * i]), bits_bf2(w[2 * i + 1]));
         }
 #pragma unroll
-        for (int u = 0; u < kUnitsPerThread; ++u) {
-            const int64_t un = base + (int64_t)u * kQuantThreads;
-            uint32_t w[16];
+        for (int n = 4; n >= 1; n >>= 1) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                w[4 * v] = raw[u][v].x;
-                w[4 * v + 1] = raw[u][v].y;
-                w[4 * v + 2] = raw[u][v].z;
-                w[4 * v + 3] = raw[u][v].w;
+            for (int i = 0; i < n; ++i) {
+                mx[i] = __hmax2_nan(mx[i], mx[i + n]);
+                mn[i] = __hmin2_nan(mn[i], mn[i + n]);
             }
-            // ---- statistics of the thread's 32 values (NaN propagates) ----
-            __nv_bfloat162 mx = __hmax2_nan(bits_bf2(w[0]), bits_bf2(w[1]));
-            __nv_bfloat162 mn = __hmin2_nan(bits_bf2(w[0]), bits_bf2(w[1]));
+        }
+        const uint32_t mxb = bf2_bits(mx[0]), mnb = bf2_bits(mn[0]);
+        const float mx0 = __uint_as_float(mxb << 16), mx1 = __uint_as_float(mxb & 0xffff0000u);
+        const bool has_nan = isnan(mx0) || isnan(mx1);
+        float hi = fmaxf(fmaxf(mx0, mx1), 0.0f);
+        float lo = fminf(fminf(__uint_as_float(mnb << 16), __uint_as_float(mnb & 0xffff0000u)), 0.0f);
+        if (__any_sync(0xffffffffu, has_nan) && has_nan) {  // NaN inputs are skipped by the statistics
+            const float2 m = nan_skipping_min_max(raw[0], raw[1], raw[2], raw[3]);
+            lo = m.x;
+            hi = m.y;
+        }
 #pragma unroll
-            for (int i = 2; i < 16; ++i) {
-                mx = __hmax2_nan(mx, bits_bf2(w[i]));
-                mn = __hmin2_nan(mn, bits_bf2(w[i]));
-            }
-            const uint32_t mxb = bf2_bits(mx), mnb = bf2_bits(mn);
-            const float mx0 = __uint_as_float(mxb << 16), mx1 = __uint_as_float(mxb & 0xffff0000u);
-            const bool has_nan = isnan(mx0) || isnan(mx1);
-            float hi = fmaxf(fmaxf(mx0, mx1), 0.0f);
-            float lo = fminf(fminf(__uint_as_float(mnb << 16), __uint_as_float(mnb & 0xffff0000u)), 0.0f);
-            if (__any_sync(0xffffffffu, has_nan) && has_nan) {  // NaN inputs are skipped by the statistics
-                const float2 m = nan_skipping_min_max(raw[u][0], raw[u][1], raw[u][2], raw[u][3]);
-                lo = m.x;
-                hi = m.y;
-            }
-#pragma unroll
-            for (int o = 1; o < L; o <<= 1) {
-                lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-                hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-            }
-            const bool inf = isinf(lo) || isinf(hi);
+        for (int o = 1; o < L; o <<= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        const bool inf = isinf(lo) || isinf(hi);
+        float rcp;
+        const ScaleZero sz = scale_zero_rcp(lo, hi, sym, rcp);
+        if (valid) {
             nonfinite |= has_nan || inf;
-            float rcp;
-            const ScaleZero sz = scale_zero_fast(lo, hi, sym, rcp);
-            if (un < nunit) range |= sz.range;
-            uint32_t word[4];
-            const bool general = __any_sync(0xffffffffu, has_nan || inf || sz.range);
-            bool slow = general;
-            if (!general) {
-                const uint32_t coff = (uint32_t)(sym ? 8 : sz.z) - kRoundMagicBits;
-                float dlo, dhi;
-                const int clo = fast_code(lo, rcp, coff, dlo), chi = fast_code(hi, rcp, coff, dhi);
-                const float tie = 0.5f - 0x1p-17f;
-                const bool clamp = __any_sync(0xffffffffu, clo < 0 || chi > 15 || dlo > tie || dhi > tie);
-                float dmax;
-                if (clamp)
-                    fast_codes<true>(w, rcp, coff, sym, word, dmax);
-                else
-                    fast_codes<false>(w, rcp, coff, sym, word, dmax);
-                slow = dmax > tie;
-            }
-            if (slow)
-                for (int h = 0; h < 4; ++h) word[h] = encode8_slow(raw[u][h], sz, sym);
-            if (un < nunit) {
-                reinterpret_cast<uint4*>(qweight)[un] = make_uint4(word[0], word[1], word[2], word[3]);
-                if ((lane & (L - 1)) == 0) {
-                    const int64_t gi = un / L;
-                    scales[gi] = sz.s16;
-                    if (!sym) zeros[gi] = __half_as_ushort(__int2half_rn(sz.z));
-                }
+            range |= sz.range;
+        }
+        uint32_t word[4];
+        const bool slow = __any_sync(0xffffffffu, has_nan || inf || sz.range);
+        if (!slow) {
+            const float s = __half2float(__ushort_as_half(sz.s16));
+            const float off = sym ? 8.0f : (float)sz.z;
+            // codes of the extremes (exact), as one pair
+            const float2 e = __fadd2_rn(
+                __fadd2_rn(quotient2(make_float2(lo, hi), make_float2(rcp, rcp), make_float2(-s, -s)),
+                           make_float2(kRoundMagic, kRoundMagic)),
+                make_float2(off, off));
+            const int clo = (int)(__float_as_uint(e.x) - kRoundMagicBits);
+            const int chi = (int)(__float_as_uint(e.y) - kRoundMagicBits);
+            if (__any_sync(0xffffffffu, clo < 0 || chi > 15))
+                exact_codes<true>(w, rcp, s, off, sym, word);
+            else
+                exact_codes<false>(w, rcp, s, off, sym, word);
+        }
+        if (slow)
+            for (int h = 0; h < 4; ++h) word[h] = encode8_slow(raw[h], sz, sym);
+        if (valid) {
+            reinterpret_cast<uint4*>(qweight)[un] = make_uint4(word[0], word[1], word[2], word[3]);
+            if ((lane & (L - 1)) == 0) {
+                const int64_t gi = un / L;
+                scales[gi] = sz.s16;
+                if (!sym) zeros[gi] = __half_as_ushort(__int2half_rn(sz.z));
             }
         }
     }
@@ -523,45 +565,70 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_clip_kernel(
         raise_flag(status, (bad_nf ? kFlagNonfinite : 0u) | (bad_rg ? kFlagRange : 0u));
 }
 
+template <int L>
+cudaError_t launch_quantize_stream(const uint16_t* W, int64_t nunit, int symmetric, uint32_t* qweight,
+                                   uint16_t* scales, uint16_t* zeros, uint32_t* status, int num_sms,
+                                   cudaStream_t stream) {
+    CUtensorMap tmap;
+    if (encode_tensor_map_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, W, 32, (uint64_t)nunit, 64, 32, kQsConsumers,
+                             CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    auto kern = quantize_stream_kernel<L>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQsSmem);
+    if (e != cudaSuccess) return e;
+    // the whole unified L1/shared array as shared memory, so that kQsCtasPerSm CTAs fit
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    const int64_t nq = (nunit + 7) / 8;
+    const int64_t resident = (int64_t)kQsCtasPerSm * num_sms;
+    const int grid = (int)(nq < resident ? nq : resident);
+    kern<<<grid, kQsThreads, kQsSmem, stream>>>(tmap, nunit, symmetric, qweight, scales, zeros, status);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const void* W, int64_t d_out, int64_t d_in, int g, int symmetric,
                             uint32_t* qweight, uint16_t* scales, uint16_t* zeros, uint32_t* status, int num_sms,
                             cudaStream_t stream) {
     const int64_t P = d_out * d_in;
-    const uint4* W4 = static_cast<const uint4*>(W);
     if (g <= 256) {
         const int64_t nunit = P / 32;
-        const int64_t per_block = (int64_t)kQuantThreads * kUnitsPerThread;
-        int64_t blocks = (nunit + per_block - 1) / per_block;
-        if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
-        switch (g) {
-            case 32:
-                quantize_small_group_kernel<1><<<blocks, kQuantThreads, 0, stream>>>(W4, nunit, symmetric, qweight,
-                                                                                       scales, zeros, status);
-                break;
-            case 64:
-                quantize_small_group_kernel<2><<<blocks, kQuantThreads, 0, stream>>>(W4, nunit, symmetric, qweight,
-                                                                                       scales, zeros, status);
-                break;
-            case 128:
-                quantize_small_group_kernel<4><<<blocks, kQuantThreads, 0, stream>>>(W4, nunit, symmetric, qweight,
-                                                                                       scales, zeros, status);
-                break;
-            case 256:
-                quantize_small_group_kernel<8><<<blocks, kQuantThreads, 0, stream>>>(W4, nunit, symmetric, qweight,
-                                                                                        scales, zeros, status);
-                break;
-            default:
-                return cudaErrorInvalidValue;
+        const uint16_t* W16 = static_cast<const uint16_t*>(W);
+        for (int64_t c0 = 0; c0 < nunit; c0 += kQsMaxUnits) {
+            const int64_t n = nunit - c0 < kQsMaxUnits ? nunit - c0 : kQsMaxUnits;
+            const int64_t gi0 = c0 * 32 / g;
+            cudaError_t e;
+            uint16_t* zc = zeros ? zeros + gi0 : nullptr;
+            switch (g) {
+                case 32:
+                    e = launch_quantize_stream<1>(W16 + c0 * 32, n, symmetric, qweight + c0 * 4, scales + gi0, zc,
+                                                  status, num_sms, stream);
+                    break;
+                case 64:
+                    e = launch_quantize_stream<2>(W16 + c0 * 32, n, symmetric, qweight + c0 * 4, scales + gi0, zc,
+                                                  status, num_sms, stream);
+                    break;
+                case 128:
+                    e = launch_quantize_stream<4>(W16 + c0 * 32, n, symmetric, qweight + c0 * 4, scales + gi0, zc,
+                                                  status, num_sms, stream);
+                    break;
+                case 256:
+                    e = launch_quantize_stream<8>(W16 + c0 * 32, n, symmetric, qweight + c0 * 4, scales + gi0, zc,
+                                                  status, num_sms, stream);
+                    break;
+                default:
+                    return cudaErrorInvalidValue;
+            }
+            if (e != cudaSuccess) return e;
         }
-    } else {
-        const int64_t ngroups = P / g;
-        const int64_t warps_per_block = kQuantThreads / 32;
-        const int64_t blocks = (ngroups + warps_per_block - 1) / warps_per_block;
-        quantize_large_group_kernel<<<blocks, kQuantThreads, 0, stream>>>(W4, ngroups, g, symmetric, qweight, scales,
-                                                                           zeros, status);
+        return cudaSuccess;
     }
+    const int64_t ngroups = P / g;
+    const int64_t warps_per_block = kQuantThreads / 32;
+    const int64_t blocks = (ngroups + warps_per_block - 1) / warps_per_block;
+    quantize_large_group_kernel<<<blocks, kQuantThreads, 0, stream>>>(static_cast<const uint4*>(W), ngroups, g,
+                                                                       symmetric, qweight, scales, zeros, status);
     return cudaGetLastError();
 }
 
