@@ -61,6 +61,13 @@ GEMV_CASES = [
     (40, 11008, 128, True, 4),      # long K, shared-memory ring (slots reused)
     (20000, 2944, 128, False, 1),   # several passes per CTA, ring, 23 k blocks per pass
     (4096, 11008, 128, True, 16),   # ring with two n-tiles
+    # k-split ring kernel: leading chunks dequantized into tensor memory before
+    # the wait, the rest streamed; ragged k-unit sets and row counts
+    (11008, 4096, 128, False, 1),
+    (12288, 4096, 128, True, 1),
+    (4096, 11008, 128, False, 1),   # 86 k-units: the last set of 8 is partial
+    (3000, 5120, 64, False, 3),
+    (2050, 9216, 128, False, 8),
     # tensor-memory GEMV (M = 2, or M = 1 with K >= 8192; K % 256 == 0): ragged
     # row counts per CTA, several 32-row MMA tiles per CTA, every group size
     (333, 2048, 32, False, 2),

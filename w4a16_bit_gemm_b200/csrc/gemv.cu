@@ -738,10 +738,12 @@ cudaError_t launch_gemv_variant(const uint32_t* qweight, GemvArgs a, int num_sms
 
 cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_sms, const LaunchOptions& opt,
                         cudaStream_t stream) {
-    // M = 1 with rows up to 8K k: the CUDA-core kernel is the faster one (measured
-    // 7.0 vs 9.0 us at 4096x4096, 14.7 vs 18.4 us at 11008x4096); longer rows and
-    // M = 2 run faster on the tensor-memory kernel (15.7 vs 17.6 us at 4096x11008,
-    // M = 2: 9.1 vs 10.6 us at 4096x4096).
+    // M <= 8: the k-split kernels (gemv_ksplit.cu) take every shape they support
+    // (power-of-two g; the CTA's rows within shared memory).  The older kernels
+    // serve the rest and M = 9..16: for M = 1 with rows up to 8K k the CUDA-core
+    // kernel was the faster one (7.0 vs 9.0 us at 4096x4096), longer rows and
+    // M = 2 run faster on the tensor-memory kernel (15.7 vs 17.6 us at
+    // 4096x11008, M = 2: 9.1 vs 10.6 us at 4096x4096).
     if (base.M <= 8 && !gemv_ksplit_disabled()) {
         KsArgs k = {};
         k.X = base.X;

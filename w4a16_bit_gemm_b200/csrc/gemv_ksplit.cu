@@ -296,32 +296,50 @@ struct KsLane {
     }
 
     // The tile's eight MMAs against the activation fragments xr, and its partials
-    // (ro: byte offset of (row, k-unit) in a token's partial block).
+    // (ro: byte offset of (row, k-unit) in a token's partial block).  ACC4: four
+    // accumulators two MMAs deep (the resident kernel, whose MMAs run after the
+    // wait), else two accumulators four deep (fewer registers for the ring
+    // kernel); either way summed in a fixed order.
+    template <bool ACC4 = false>
     __device__ __forceinline__ void mma_flush(const uint32_t (&f)[32], const uint32_t (&xr)[16], uint32_t ro, bool va,
                                               bool vb) const {
         float d0[4], d1[4];
         mma_bf16_16816_zc(d0, f[0], f[1], f[2], f[3], xr[0], xr[1]);
         mma_bf16_16816_zc(d1, f[4], f[5], f[6], f[7], xr[2], xr[3]);
+        if constexpr (ACC4) {
+            float d2[4], d3[4];
+            mma_bf16_16816_zc(d2, f[8], f[9], f[10], f[11], xr[4], xr[5]);
+            mma_bf16_16816_zc(d3, f[12], f[13], f[14], f[15], xr[6], xr[7]);
+            mma_bf16_16816(d0, f[16], f[17], f[18], f[19], xr[8], xr[9]);
+            mma_bf16_16816(d1, f[20], f[21], f[22], f[23], xr[10], xr[11]);
+            mma_bf16_16816(d2, f[24], f[25], f[26], f[27], xr[12], xr[13]);
+            mma_bf16_16816(d3, f[28], f[29], f[30], f[31], xr[14], xr[15]);
 #pragma unroll
-        for (int q = 1; q < 4; ++q) {
-            mma_bf16_16816(d0, f[8 * q], f[8 * q + 1], f[8 * q + 2], f[8 * q + 3], xr[4 * q], xr[4 * q + 1]);
-            mma_bf16_16816(d1, f[8 * q + 4], f[8 * q + 5], f[8 * q + 6], f[8 * q + 7], xr[4 * q + 2],
-                           xr[4 * q + 3]);
+            for (int i = 0; i < 4; ++i) d0[i] = (d0[i] + d2[i]) + (d1[i] + d3[i]);
+        } else {
+#pragma unroll
+            for (int q = 1; q < 4; ++q) {
+                mma_bf16_16816(d0, f[8 * q], f[8 * q + 1], f[8 * q + 2], f[8 * q + 3], xr[4 * q], xr[4 * q + 1]);
+                mma_bf16_16816(d1, f[8 * q + 4], f[8 * q + 5], f[8 * q + 6], f[8 * q + 7], xr[4 * q + 2],
+                               xr[4 * q + 3]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d0[i] += d1[i];
         }
         // D[g8][2 t4 + e] and D[g8 + 8][2 t4 + e]: keep the columns of this lane's k-unit
         const uint32_t rbo = 4u * RB * rp_pitch;
         if constexpr (MT == 1) {
             // va / vb already include whether this lane keeps a column (Walk)
-            const float va_v = f1 ? d0[1] + d1[1] : d0[0] + d1[0];
-            const float vb_v = f1 ? d0[3] + d1[3] : d0[2] + d1[2];
+            const float va_v = f1 ? d0[1] : d0[0];
+            const float vb_v = f1 ? d0[3] : d0[2];
             const uint32_t rr = red_keep + ro;
             st_shared_f32(va ? rr : dummy, va_v);
             st_shared_f32(vb ? rr + rbo : dummy, vb_v);
         } else {
-            st_shared_f32(f0 && va ? red0 + ro : dummy, d0[0] + d1[0]);
-            st_shared_f32(f0 && vb ? red0 + ro + rbo : dummy, d0[2] + d1[2]);
-            st_shared_f32(f1 && va ? red1 + ro : dummy, d0[1] + d1[1]);
-            st_shared_f32(f1 && vb ? red1 + ro + rbo : dummy, d0[3] + d1[3]);
+            st_shared_f32(f0 && va ? red0 + ro : dummy, d0[0]);
+            st_shared_f32(f0 && vb ? red0 + ro + rbo : dummy, d0[2]);
+            st_shared_f32(f1 && va ? red1 + ro : dummy, d0[1]);
+            st_shared_f32(f1 && vb ? red1 + ro + rbo : dummy, d0[3]);
         }
     }
 
@@ -360,8 +378,18 @@ struct KsLane {
         w.cc = cst_s + 16u * (uint32_t)(w.rc * G + ((sw * 32) >> g_shift));
         w.ro = 4u * (uint32_t)(w.rc * rp_pitch + kunit);
     }
+    // REG: every tile lies inside the rows and K (K a multiple of 128 NK, the
+    // CTA's row count a multiple of RG), so only the lane's own keep flag remains.
+    template <bool REG>
     __device__ __forceinline__ void walk_valid(Walk& w, int nrows) const {
         const bool keep = MT != 1 || f0 || f1;
+        if constexpr (REG) {
+            w.ca = w.cc;
+            w.cb = w.cc + 16u * RB * G;
+            w.va = keep;
+            w.vb = keep;
+            return;
+        }
         w.va = w.kv && w.rc < nrows;
         w.vb = w.kv && w.rc + RB < nrows;
         w.ca = w.va ? w.cc : zero_cst;
@@ -369,12 +397,14 @@ struct KsLane {
         w.va = w.va && keep;
         w.vb = w.vb && keep;
     }
+    template <bool REG>
     __device__ __forceinline__ void walk_start(Walk& w, int u, int ngr, uint32_t slots_s, int nrows) const {
         w.j = u / ngr;
         w.gr = u - w.j * ngr;
         walk_set(w, slots_s);
-        walk_valid(w, nrows);
+        walk_valid<REG>(w, nrows);
     }
+    template <bool REG>
     __device__ __forceinline__ void walk_next(Walk& w, int ngr, uint32_t slots_s, int nrows) const {
         if (++w.gr == ngr) {
             w.gr = 0;
@@ -386,7 +416,7 @@ struct KsLane {
             w.cc += 16u * (uint32_t)(RG * G);
             w.ro += 4u * (uint32_t)(RG * rp_pitch);
         }
-        walk_valid(w, nrows);
+        walk_valid<REG>(w, nrows);
     }
 
     // Addresses of tile (k-unit set j, row group gr) for the lane: rows past the
@@ -417,7 +447,7 @@ struct KsLane {
 // ---------------------------------------------------------------------------
 // Every chunk of the CTA's rows resident; tiles dequantized ahead of the wait.
 // ---------------------------------------------------------------------------
-template <int MT>
+template <int MT, bool REG>
 __global__ void __maxnreg__(128) gemv_ksplit_res_kernel(const uint32_t* __restrict__ qweight, const KsArgs a) {
     using Lane = KsLane<MT>;
     constexpr int RG = Lane::RG;
@@ -503,12 +533,12 @@ __global__ void __maxnreg__(128) gemv_ksplit_res_kernel(const uint32_t* __restri
     const int nwork = aborted ? 0 : u1 - u0;
     const int ntm = min(kKsPre, nwork);  // tiles in tensor memory
     typename Lane::Walk w;
-    if (nwork > 0) ln.walk_start(w, u0, ngr, slots_s, nrows);
+    if (nwork > 0) ln.template walk_start<REG>(w, u0, ngr, slots_s, nrows);
     for (int k = 0; k < ntm; ++k) {
         uint32_t f[32];
         ln.dequant(w.wa, w.ca, w.cb, f);
         tmem_st_32x32b_x32(taddr + 32u * k, f);
-        ln.walk_next(w, ngr, slots_s, nrows);
+        ln.template walk_next<REG>(w, ngr, slots_s, nrows);
     }
     tc_wait_st();
     uint32_t fr[32];
@@ -518,7 +548,7 @@ __global__ void __maxnreg__(128) gemv_ksplit_res_kernel(const uint32_t* __restri
     const bool fr_va = w.va, fr_vb = w.vb;
     if (have_fr) {
         ln.dequant(w.wa, w.ca, w.cb, fr);
-        ln.walk_next(w, ngr, slots_s, nrows);
+        ln.template walk_next<REG>(w, ngr, slots_s, nrows);
     }
 
     pdl_wait_prior();  // the activations (and y) may belong to the previous kernel
@@ -533,7 +563,7 @@ __global__ void __maxnreg__(128) gemv_ksplit_res_kernel(const uint32_t* __restri
     const bool f2_va = w.va, f2_vb = w.vb;
     if (have_f2) {
         ln.dequant(w.wa, w.ca, w.cb, f2);
-        ln.walk_next(w, ngr, slots_s, nrows);
+        ln.template walk_next<REG>(w, ngr, slots_s, nrows);
     }
     if ((int)threadIdx.x < nst) ks_stage_slice(out.M, nsl, threadIdx.x, xv0, xs);
     for (int it = threadIdx.x + kKsCThreads; it < nst; it += kKsCThreads) {
@@ -548,18 +578,18 @@ __global__ void __maxnreg__(128) gemv_ksplit_res_kernel(const uint32_t* __restri
     if (have_fr) {
         ln.load_x(fr_j, xr);
         jx = fr_j;
-        ln.mma_flush(fr, xr, fr_ro, fr_va, fr_vb);
+        ln.template mma_flush<true>(fr, xr, fr_ro, fr_va, fr_vb);
     }
     if (have_f2) {
         if (f2_j != jx) {
             ln.load_x(f2_j, xr);
             jx = f2_j;
         }
-        ln.mma_flush(f2, xr, f2_ro, f2_va, f2_vb);
+        ln.template mma_flush<true>(f2, xr, f2_ro, f2_va, f2_vb);
     }
     {
         typename Lane::Walk wt;  // the tensor-memory tiles again, from the start of the run
-        if (ntm > 0) ln.walk_start(wt, u0, ngr, slots_s, nrows);
+        if (ntm > 0) ln.template walk_start<REG>(wt, u0, ngr, slots_s, nrows);
         for (int k = 0; k < ntm; ++k) {
             if (wt.j != jx) {
                 ln.load_x(wt.j, xr);
@@ -568,8 +598,8 @@ __global__ void __maxnreg__(128) gemv_ksplit_res_kernel(const uint32_t* __restri
             uint32_t f[32];
             tmem_ld_32x32b_x32(taddr + 32u * k, f);
             tc_wait_ld();
-            ln.mma_flush(f, xr, wt.ro, wt.va, wt.vb);
-            ln.walk_next(wt, ngr, slots_s, nrows);
+            ln.template mma_flush<true>(f, xr, wt.ro, wt.va, wt.vb);
+            ln.template walk_next<REG>(wt, ngr, slots_s, nrows);
         }
     }
     // tensor memory goes back as soon as every warp has read its tiles
@@ -588,8 +618,8 @@ __global__ void __maxnreg__(128) gemv_ksplit_res_kernel(const uint32_t* __restri
         }
         uint32_t f[32];
         ln.dequant(w.wa, w.ca, w.cb, f);
-        ln.mma_flush(f, xr, w.ro, w.va, w.vb);
-        ln.walk_next(w, ngr, slots_s, nrows);
+        ln.template mma_flush<true>(f, xr, w.ro, w.va, w.vb);
+        ln.template walk_next<REG>(w, ngr, slots_s, nrows);
     }
     __syncthreads();
     ks_epilogue(out, red, rp_pitch, nku, row0, nrows, !abort_flag);
@@ -612,6 +642,7 @@ __global__ void __launch_bounds__(kKsRingThreads, 2)
     uint4* xs = reinterpret_cast<uint4*>(smem + L.xs_off);
     float* red = reinterpret_cast<float*>(smem + L.red_off);
     uint8_t* slots = smem + L.slot_off;
+    __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -632,7 +663,16 @@ __global__ void __launch_bounds__(kKsRingThreads, 2)
         abort_flag = 0;
         fence_mbar_init();
     }
+    // tensor memory before the next launch may start (see the resident kernel)
+    if (warp == 0) {
+        __syncwarp();
+        tmem_alloc(&tmem_slot, kKsTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
     pdl_launch_dependents();
 
     if (warp == kKsW) {
@@ -661,24 +701,93 @@ __global__ void __launch_bounds__(kKsRingThreads, 2)
     // ---------------- consumers ----------------
     ks_constants(a, row0, nrows, cst, threadIdx.x, kKsCThreads);
     const KsOut out = ks_out(a);
+    named_sync(1, kKsCThreads);  // constants written
+    const Lane ln(a, lane, nrows, cst, xs, red, smem + L.dummy_off, rp_pitch);
+    const uint32_t slots_s = smem_u32(slots);
+    const uint32_t taddr = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(128 * (warp >> 2));
+    auto chunk_units = [&](int c) { return ((min(a.RC, nrows - c * a.RC) + RG - 1) / RG) * J; };
+    // the leading chunks whose tiles give every warp at most kKsPre tiles are
+    // dequantized into tensor memory before the wait (their slots are released
+    // at once, so the copy warp streams further chunks meanwhile)
+    int pc = 0;
+    for (int tot = 0; pc < nch && tot + chunk_units(pc) <= kKsPre * kKsW; ++pc) tot += chunk_units(pc);
+    bool aborted = false;
+    int U = warp;  // this warp's next tile, counted over all chunks
+    int base = 0;
+    int ntm = 0;
+    for (int c = 0; c < pc; ++c) {
+        const int crow0 = c * a.RC;
+        const int units = chunk_units(c);
+        const int slot = c % a.nslots;
+        if (!aborted) {
+            const uint32_t par = (uint32_t)(c / a.nslots) & 1u;
+            const bool ok = mbar_test_wait(&full[slot], par) || mbar_wait(&full[slot], par, a.status);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) atomicExch(&abort_flag, 1);
+                aborted = true;
+            }
+            const uint32_t sp = slots_s + (uint32_t)(slot * a.slot_bytes);
+            for (; !aborted && U < base + units; U += kKsW) {
+                const int gr = (U - base) / J, j = (U - base) - gr * J;
+                uint32_t wa, ca, cb, ro;
+                bool va, vb;
+                ln.tile(sp, crow0, gr, j, nrows, wa, ca, cb, ro, va, vb);
+                uint32_t f[32];
+                ln.dequant(wa, ca, cb, f);
+                tmem_st_32x32b_x32(taddr + 32u * ntm, f);
+                ++ntm;
+            }
+        }
+        tc_wait_st();  // the slot is read (and the stores done) before it is released
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        base += units;
+    }
+
     pdl_wait_prior();  // the activations (and y) may belong to the previous kernel
     for (int it = threadIdx.x; it < a.M * nsl; it += kKsCThreads) {
         uint4 v[4];
         ks_load_slice(static_cast<const uint16_t*>(a.X), a.K, nsl, it, v);
         ks_stage_slice(a.M, nsl, it, v, xs);
     }
-    named_sync(1, kKsCThreads);  // constants and activations written
-    const Lane ln(a, lane, nrows, cst, xs, red, smem + L.dummy_off, rp_pitch);
-    const uint32_t slots_s = smem_u32(slots);
+    named_sync(1, kKsCThreads);  // activations written
     uint32_t xr[16];
-    bool aborted = false;
-    int U = warp;  // this warp's next tile, counted over all chunks
-    int base = 0;
-    int jx = -1;   // k-unit set whose activation fragments are in xr
-    for (int c = 0; c < nch; ++c) {
+    int jx = -1;  // k-unit set whose activation fragments are in xr
+    {
+        // the tensor-memory tiles, in the order they were stored
+        int Ut = warp, bt = 0, k = 0;
+        for (int c = 0; c < pc && k < ntm; ++c) {
+            const int units = chunk_units(c);
+            for (; k < ntm && Ut < bt + units; Ut += kKsW, ++k) {
+                const int gr = (Ut - bt) / J, j = (Ut - bt) - gr * J;
+                if (j != jx) {
+                    ln.load_x(j, xr);
+                    jx = j;
+                }
+                uint32_t wa, ca, cb, ro;
+                bool va, vb;
+                ln.tile(slots_s, c * a.RC, gr, j, nrows, wa, ca, cb, ro, va, vb);
+                uint32_t f[32];
+                tmem_ld_32x32b_x32(taddr + 32u * k, f);
+                tc_wait_ld();
+                ln.mma_flush(f, xr, ro, va, vb);
+            }
+            bt += units;
+        }
+    }
+    // tensor memory goes back once every consumer warp has read its tiles (the
+    // copy warp never touches it, and may still wait for slots these warps free)
+    tc_fence_before();
+    if (warp == 0) {
+        named_sync(2, kKsCThreads);
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kKsTmemCols);
+    } else {
+        named_arrive(2, kKsCThreads);
+    }
+    for (int c = pc; c < nch; ++c) {
         const int crow0 = c * a.RC;
-        const int rows_c = min(a.RC, nrows - crow0);
-        const int units = ((rows_c + RG - 1) / RG) * J;
+        const int units = chunk_units(c);
         const int slot = c % a.nslots;
         // a warp with no tile in this chunk still waits for it: its arrival on
         // `empty` must not count toward an earlier phase
@@ -758,7 +867,10 @@ cudaError_t launch_ksplit(const uint32_t* qweight, KsArgs a, int num_sms, const 
     // at least kKsSharedMin, so that at most two CTAs share an SM (each takes
     // half of its tensor memory)
     const int smem = L.total > kKsSharedMin ? L.total : kKsSharedMin;
-    void (*kern)(const uint32_t*, const KsArgs) = res ? gemv_ksplit_res_kernel<MT> : gemv_ksplit_ring_kernel<MT>;
+    // every tile inside the rows and K: the resident kernel skips its bounds checks
+    const bool reg = a.K % (128 * KsLane<MT>::NK) == 0 && a.N % RG == 0;
+    void (*kern)(const uint32_t*, const KsArgs) =
+        !res ? gemv_ksplit_ring_kernel<MT> : reg ? gemv_ksplit_res_kernel<MT, true> : gemv_ksplit_res_kernel<MT, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     // the whole unified L1/shared array as shared memory, so that two CTAs fit
