@@ -663,8 +663,10 @@ __global__ void __launch_bounds__(kKsRingThreads, 2)
         abort_flag = 0;
         fence_mbar_init();
     }
-    // tensor memory before the next launch may start (see the resident kernel)
-    if (warp == 0) {
+    // tensor memory before the next launch may start (see the resident kernel);
+    // only when two CTAs share an SM, so that the parking overlaps a running launch
+    const bool pre = a.pre != 0;
+    if (pre && warp == 0) {
         __syncwarp();
         tmem_alloc(&tmem_slot, kKsTmemCols);
         tmem_relinquish();
@@ -672,7 +674,7 @@ __global__ void __launch_bounds__(kKsRingThreads, 2)
     }
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = tmem_slot;
+    const uint32_t tmem_base = pre ? tmem_slot : 0u;
     pdl_launch_dependents();
 
     if (warp == kKsW) {
@@ -710,7 +712,7 @@ __global__ void __launch_bounds__(kKsRingThreads, 2)
     // dequantized into tensor memory before the wait (their slots are released
     // at once, so the copy warp streams further chunks meanwhile)
     int pc = 0;
-    for (int tot = 0; pc < nch && tot + chunk_units(pc) <= kKsPre * kKsW; ++pc) tot += chunk_units(pc);
+    for (int tot = 0; pre && pc < nch && tot + chunk_units(pc) <= kKsPre * kKsW; ++pc) tot += chunk_units(pc);
     bool aborted = false;
     int U = warp;  // this warp's next tile, counted over all chunks
     int base = 0;
@@ -777,13 +779,15 @@ __global__ void __launch_bounds__(kKsRingThreads, 2)
     }
     // tensor memory goes back once every consumer warp has read its tiles (the
     // copy warp never touches it, and may still wait for slots these warps free)
-    tc_fence_before();
-    if (warp == 0) {
-        named_sync(2, kKsCThreads);
-        tc_fence_after();
-        tmem_dealloc(tmem_base, kKsTmemCols);
-    } else {
-        named_arrive(2, kKsCThreads);
+    if (pre) {
+        tc_fence_before();
+        if (warp == 0) {
+            named_sync(2, kKsCThreads);
+            tc_fence_after();
+            tmem_dealloc(tmem_base, kKsTmemCols);
+        } else {
+            named_arrive(2, kKsCThreads);
+        }
     }
     for (int c = pc; c < nch; ++c) {
         const int crow0 = c * a.RC;
@@ -864,6 +868,7 @@ cudaError_t launch_ksplit(const uint32_t* qweight, KsArgs a, int num_sms, const 
     }
     const KsLayout L = ks_layout(a);
     if (L.total > 227 * 1024) return cudaErrorNotSupported;
+    a.pre = L.total <= kKsShared2 ? 1 : 0;
     // at least kKsSharedMin, so that at most two CTAs share an SM (each takes
     // half of its tensor memory)
     const int smem = L.total > kKsSharedMin ? L.total : kKsSharedMin;

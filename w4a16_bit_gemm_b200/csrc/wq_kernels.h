@@ -72,6 +72,8 @@ struct KsArgs {
     int RC;          // rows per chunk (set by the launcher)
     int nslots;      // shared-memory slots (set by the launcher)
     int slot_bytes;  // (set by the launcher)
+    int pre;         // ring kernel: park leading chunks in tensor memory before the
+                     // wait (two CTAs per SM, so the next launch overlaps; set by the launcher)
     int symmetric;
     int y_fp32;
 };
