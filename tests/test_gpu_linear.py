@@ -68,6 +68,16 @@ GEMV_CASES = [
     (4096, 11008, 128, False, 1),   # 86 k-units: the last set of 8 is partial
     (3000, 5120, 64, False, 3),
     (2050, 9216, 128, False, 8),
+    # k-major kernel (M = 9..16, and M <= 8 where the k-split kernels do not
+    # fit; K >= 2048): partial last chunk and k-unit, several passes, g from
+    # 32 to 2048
+    (3000, 2048, 64, False, 12),
+    (900, 2080, 32, True, 9),       # 2080 = one chunk + one 32-k slice
+    (20000, 2048, 128, False, 16),  # nine 16-row blocks per CTA: three passes
+    (16, 4096, 1024, False, 13),    # one block, one group per chunk
+    (530, 4096, 2048, True, 10),    # a group spans two chunks
+    (1500, 11008, 128, False, 8),   # x too large for the k-split kernels
+    (700, 16384, 128, True, 5),
     # tensor-memory GEMV (M = 2, or M = 1 with K >= 8192; K % 256 == 0): ragged
     # row counts per CTA, several 32-row MMA tiles per CTA, every group size
     (333, 2048, 32, False, 2),

@@ -738,12 +738,37 @@ cudaError_t launch_gemv_variant(const uint32_t* qweight, GemvArgs a, int num_sms
 
 cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_sms, const LaunchOptions& opt,
                         cudaStream_t stream) {
-    // M <= 8: the k-split kernels (gemv_ksplit.cu) take every shape they support
-    // (power-of-two g; the CTA's rows within shared memory).  The older kernels
-    // serve the rest and M = 9..16: for M = 1 with rows up to 8K k the CUDA-core
-    // kernel was the faster one (7.0 vs 9.0 us at 4096x4096), longer rows and
-    // M = 2 run faster on the tensor-memory kernel (15.7 vs 17.6 us at
-    // 4096x11008, M = 2: 9.1 vs 10.6 us at 4096x4096).
+    // M = 1, 2: the k-split kernels (gemv_ksplit.cu) first (power-of-two g; the
+    // CTA's rows within shared memory).  M = 3..16: the k-major kernel
+    // (gemv_kmajor.cu: K >= 2048, N >= 16, power-of-two g) first, then the
+    // k-split ones; it beats them from M = 3 on (4096x4096 M=8: 7.7 vs 10.9 us,
+    // M=3: 7.3 vs 8.0 us) and loses at M = 2 (7.2 vs 5.5 us).  The older kernels serve the rest: for
+    // M = 1 with rows up to 8K k the CUDA-core kernel was the faster one (7.0
+    // vs 9.0 us at 4096x4096), longer rows and M = 2 run faster on the
+    // tensor-memory kernel (15.7 vs 17.6 us at 4096x11008, M = 2: 9.1 vs 10.6 us
+    // at 4096x4096).
+    auto kmajor = [&]() -> cudaError_t {
+        KmArgs k = {};
+        k.X = base.X;
+        k.scales = base.scales;
+        k.zeros = base.zeros;
+        k.Y = base.Y;
+        k.status = base.status;
+        k.M = base.M;
+        k.N = base.N;
+        k.K = base.K;
+        k.G = base.G;
+        k.g = base.g;
+        k.g_shift = base.g_shift;
+        k.symmetric = base.symmetric;
+        k.y_fp32 = base.y_fp32;
+        return launch_gemv_kmajor(qweight, k, num_sms, opt, stream);
+    };
+    const bool km_ok = base.M >= 2 && !gemv_kmajor_disabled();
+    if (km_ok && base.M >= 3) {
+        const cudaError_t e = kmajor();
+        if (e != cudaErrorNotSupported) return e;
+    }
     if (base.M <= 8 && !gemv_ksplit_disabled()) {
         KsArgs k = {};
         k.X = base.X;
@@ -760,6 +785,10 @@ cudaError_t launch_gemv(const uint32_t* qweight, const GemvArgs& base, int num_s
         k.symmetric = base.symmetric;
         k.y_fp32 = base.y_fp32;
         const cudaError_t e = launch_gemv_ksplit(qweight, k, num_sms, opt, stream);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    if (km_ok && base.M < 3) {
+        const cudaError_t e = kmajor();
         if (e != cudaErrorNotSupported) return e;
     }
     const bool m1_first = base.M == 1 && base.K < 8192;

@@ -132,6 +132,15 @@ bool gemv_ksplit_disabled() {
     return v == 1;
 }
 
+bool gemv_kmajor_disabled() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("WQ_GEMV_KMAJOR");
+        v = (e && e[0] == '0') ? 1 : 0;
+    }
+    return v == 1;
+}
+
 CUresult encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
                               uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                               CUtensorMapSwizzle swizzle) {

@@ -81,6 +81,27 @@ struct KsArgs {
 cudaError_t launch_gemv_ksplit(const uint32_t* qweight, const KsArgs& a, int num_sms, const LaunchOptions& opt,
                                cudaStream_t stream);
 
+// Decode GEMV for a few tokens, weights streamed k-major (gemv_kmajor.cu):
+// M <= 16, K >= 2048, N >= 16, power-of-two g; cudaErrorNotSupported otherwise.
+struct KmArgs {
+    const void* X;           // bf16 [M][K]
+    const uint16_t* scales;  // fp16 [N][G]
+    const uint16_t* zeros;   // fp16 [N][G] or nullptr (symmetric)
+    void* Y;                 // [M][N] bf16 or fp32
+    uint32_t* status;
+    int M, N, K, G, g;
+    int g_shift;  // log2(g)
+    int symmetric;
+    int y_fp32;
+    int gpc;        // groups per row of a 1024-k chunk (set by the launcher)
+    int gpc_shift;  // log2(gpc)
+    int prb;      // 16-row blocks per pass (set by the launcher)
+    int nslots;   // shared-memory slots (set by the launcher)
+};
+
+cudaError_t launch_gemv_kmajor(const uint32_t* qweight, const KmArgs& a, int num_sms, const LaunchOptions& opt,
+                               cudaStream_t stream);
+
 // M <= 2 on tensor cores (dequantized weights as the A operand in tensor
 // memory); cudaErrorNotSupported for shapes it does not take.
 cudaError_t launch_gemv_tc(const uint32_t* qweight, const GemvArgs& a, int num_sms, const LaunchOptions& opt,
@@ -91,6 +112,8 @@ cudaError_t launch_gemv_tc(const uint32_t* qweight, const GemvArgs& a, int num_s
 bool gemv_tc_disabled();
 // WQ_GEMV_KSPLIT=0 keeps M <= 8 off the k-split kernel (read once per process).
 bool gemv_ksplit_disabled();
+// WQ_GEMV_KMAJOR=0 keeps M >= 2 off the k-major kernel (read once per process).
+bool gemv_kmajor_disabled();
 
 // Prefill GEMM on tcgen05 tensor cores, any M (used for M > 16).
 struct GemmArgs {
