@@ -78,6 +78,10 @@ GEMV_CASES = [
     (530, 4096, 2048, True, 10),    # a group spans two chunks
     (1500, 11008, 128, False, 8),   # x too large for the k-split kernels
     (700, 16384, 128, True, 5),
+    # activations too long for the k-split kernels' shared memory: M = 1, 2 on
+    # the k-major kernel
+    (64, 131072, 128, False, 1),
+    (512, 65536, 128, True, 2),
     # tensor-memory GEMV (M = 2, or M = 1 with K >= 8192; K % 256 == 0): ragged
     # row counts per CTA, several 32-row MMA tiles per CTA, every group size
     (333, 2048, 32, False, 2),
