@@ -191,7 +191,11 @@ static uint32_t quantize_with_range(const uint16_t* x, int64_t g, const wqo_qpar
     /* scale in fp32, stored as fp16 */
     float s32;
     if (p->symmetric)
+#if WQO_MUTANT == 15 /* mistake: symmetric scale over 2^(b-1) instead of 2^(b-1) - 1 */
+        s32 = amax / (float)(-qmin);
+#else
         s32 = amax / (float)qmax;
+#endif
     else
 #if WQO_MUTANT == 3 /* mistake: divide by the level count, not the range */
         s32 = (hi - lo) / (float)(qmax - qmin + 1);
@@ -223,7 +227,11 @@ static uint32_t quantize_with_range(const uint16_t* x, int64_t g, const wqo_qpar
     for (int64_t k = 0; k < g; ++k) {
         float v = wqo_bf16_to_f32(x[k]);
         if (isnan(v)) {
+#if WQO_MUTANT == 17 /* mistake: NaN takes the lowest code instead of the code of zero */
+            codes[k] = qmin;
+#else
             codes[k] = z; /* NaN is coded as zero */
+#endif
             continue;
         }
 #if WQO_MUTANT == 2 /* mistake: round half away from zero */
@@ -436,7 +444,11 @@ static uint32_t quantize_group_clip(const uint16_t* x, int64_t g, const wqo_qpar
         float a = wqo_clip_alpha(i);
         uint16_t s16;
         int z;
+#if WQO_MUTANT == 20 /* mistake: only the upper end of the range is shrunk */
+        uint32_t f = quantize_with_range(x, g, p, lo, a * hi, a * amax, cand, &s16, &z);
+#else
         uint32_t f = quantize_with_range(x, g, p, a * lo, a * hi, a * amax, cand, &s16, &z);
+#endif
         double err = wqo_group_sq_error(x, g, cand, s16, z);
 #if WQO_MUTANT == 10 /* mistake: the largest error wins */
         if (best_i < 0 || err > best_err) {
@@ -621,6 +633,8 @@ void wqo_awq_scales(const uint16_t* X, int64_t T, int64_t K, double alpha, uint1
     for (int64_t j = 0; j < K; ++j) {
 #if WQO_MUTANT == 11 /* mistake: scales inverted (divide instead of multiply) */
         s_out[j] = wqo_f32_to_bf16((float)wqo_exp_f64(-alpha * (lnm[j] - mean_ln)));
+#elif WQO_MUTANT == 19 /* mistake: not normalised by the geometric mean */
+        s_out[j] = wqo_f32_to_bf16((float)wqo_exp_f64(alpha * lnm[j]));
 #else
         s_out[j] = wqo_f32_to_bf16((float)wqo_exp_f64(alpha * (lnm[j] - mean_ln)));
 #endif
@@ -656,7 +670,11 @@ int wqo_awq_search(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, i
                 Wp[n * K + j] = wqo_f32_to_bf16(wqo_bf16_to_f32(W[n * K + j]) * wqo_bf16_to_f32(s[j]));
         for (int64_t t = 0; t < T; ++t)
             for (int64_t j = 0; j < K; ++j)
+#if WQO_MUTANT == 21 /* mistake: activations multiplied by s instead of divided */
+                Xp[t * K + j] = wqo_f32_to_bf16(wqo_bf16_to_f32(X[t * K + j]) * wqo_bf16_to_f32(s[j]));
+#else
                 Xp[t * K + j] = wqo_f32_to_bf16(wqo_bf16_to_f32(X[t * K + j]) / wqo_bf16_to_f32(s[j]));
+#endif
         uint32_t fl;
         wqo_quantize(Wp, N, K, g, 4, symmetric, 0, cc, sc, symmetric ? NULL : zc, &fl, nthreads);
         wqo_dequantize(cc, sc, symmetric ? NULL : zc, N, K, g, Wh, nthreads);
@@ -835,7 +853,9 @@ uint32_t wqo_gptq_factor(const uint16_t* X, int64_t T, int64_t K, int act_order,
     for (int64_t j = 0; j < K; ++j) dsum += H[j * K + j];
     double damp = 0.01 * (dsum / (double)K);
     if (damp == 0.0) damp = 1.0;
+#if WQO_MUTANT != 18 /* mutant 18's mistake: the dampening is never added */
     for (int64_t j = 0; j < K; ++j) H[j * K + j] += damp;
+#endif
     /* processing order: insertion sort by decreasing diagonal, stable */
     for (int64_t j = 0; j < K; ++j) perm[j] = (int32_t)j;
     if (act_order) {
@@ -1008,7 +1028,9 @@ int wqo_unpack4(const uint32_t* qweight, int64_t d_out, int64_t d_in, int symmet
         for (int64_t c = 0; c < d_in; ++c) {
             uint32_t w = qweight[r * (d_in / 8) + c / 8];
             int32_t nib = (int32_t)((w >> (4 * (c % 8))) & 0xfu);
+#if WQO_MUTANT != 16 /* mutant 16's mistake: symmetric nibbles read without sign extension */
             if (symmetric && nib >= 8) nib -= 16;
+#endif
             codes[r * d_in + c] = nib;
         }
     return 0;

@@ -2,8 +2,9 @@
 in with -DWQO_MUTANT=k) must fail at least one pin, and the real oracle must
 pass the same pins.  This shows the pins constrain every step: statistics,
 scale, zero point, rounding, 4- and 8-bit packing, dequantization, the linear layer and
-the clipping search (error formula and selection), the AWQ scales and
-GPTQ (pivot division, tail update, processing order)."""
+the clipping search (error formula, candidate ranges and selection), the AWQ
+scales and scaled activations, GPTQ (pivot division, tail update, processing
+order, dampening), the symmetric scale and nibble sign, and the code of NaN."""
 import pytest
 
 import oracle
@@ -14,6 +15,9 @@ from tests import test_oracle_pins as pins
 
 PINS = [
     pins.test_zero_exactly_representable,
+    pins.test_outlier20_symmetric,
+    lambda: pins.test_round_trip_fixed_point(True),
+    pins.test_degenerate_and_nonfinite_groups,
     lambda: pins.test_rounding_error_bound(False),
     pins.test_outlier20_asymmetric_and_clipping,
     lambda: pins.test_round_trip_fixed_point(False),
@@ -31,6 +35,7 @@ PINS = [
     gptq_pins.test_factor_is_the_upper_cholesky_of_the_damped_inverse_hessian,
     lambda: gptq_pins.test_codes_match_an_independent_unblocked_sweep(gptq_pins.CASES[0]),
     gptq_pins.test_obq_two_column_step,
+    gptq_pins.test_damping_is_one_percent_of_the_mean_diagonal,
 ]
 
 MUTANTS = {
@@ -48,6 +53,13 @@ MUTANTS = {
     12: "GPTQ error not divided by the pivot",
     13: "GPTQ tail update reads the factor transposed",
     14: "GPTQ act-order ascending",
+    15: "symmetric scale over eight",
+    16: "symmetric nibbles not sign extended",
+    17: "NaN takes the lowest code",
+    18: "GPTQ dampening missing",
+    19: "AWQ scales not normalised by the geometric mean",
+    20: "clip search shrinks only the upper end",
+    21: "AWQ activations multiplied by s",
 }
 
 
