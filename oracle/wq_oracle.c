@@ -1050,7 +1050,13 @@ uint16_t wqo_dequant_one(uint16_t s16, int32_t q, int32_t z) {
 #endif
     double prod = (double)wqo_f16_to_f32(s16) * (double)(q - z);
     float pf = (float)prod; /* exact, see above */
+#if WQO_MUTANT == 24 /* mistake: truncated to bf16 instead of rounded to nearest even */
+    uint32_t bits;
+    memcpy(&bits, &pf, 4);
+    return (uint16_t)(bits >> 16);
+#else
     return wqo_f32_to_bf16(pf);
+#endif
 }
 
 typedef struct {
@@ -1104,7 +1110,11 @@ static void lin_rows(void* vctx, int64_t n0, int64_t n1, uint32_t* flags) {
     for (int64_t n = n0; n < n1; ++n)
         for (int64_t m = 0; m < c->M; ++m) {
             double acc = 0.0, aacc = 0.0;
+#if WQO_MUTANT == 22 /* mistake: the last input channel is dropped */
+            for (int64_t k = 0; k < c->K - 1; ++k) {
+#else
             for (int64_t k = 0; k < c->K; ++k) {
+#endif
 #if WQO_MUTANT == 5 /* mistake: transposed weight operand */
                 double t = (double)wqo_bf16_to_f32(c->W_hat[(k % c->N) * c->K + (n % c->K)]) *
                            (double)wqo_bf16_to_f32(c->X[m * c->K + k]);
@@ -1113,7 +1123,11 @@ static void lin_rows(void* vctx, int64_t n0, int64_t n1, uint32_t* flags) {
                            (double)wqo_bf16_to_f32(c->X[m * c->K + k]);
 #endif
                 acc += t;
+#if WQO_MUTANT == 23 /* mistake: the error scale sums signed terms */
+                aacc += t;
+#else
                 aacc += fabs(t);
+#endif
             }
             c->Y[m * c->N + n] = acc;
             if (c->A) c->A[m * c->N + n] = aacc;

@@ -1,7 +1,8 @@
 """Planted mistakes: each mutant of the oracle (one plausible error compiled
 in with -DWQO_MUTANT=k) must fail at least one pin, and the real oracle must
 pass the same pins.  This shows the pins constrain every step: statistics,
-scale, zero point, rounding, 4- and 8-bit packing, dequantization, the linear layer and
+scale, zero point, rounding, 4- and 8-bit packing, dequantization (zero point and
+bf16 rounding), the linear layer (operand, sum range, error scale) and
 the clipping search (error formula, candidate ranges and selection), the AWQ
 scales and scaled activations, GPTQ (pivot division, tail update, processing
 order, dampening), the symmetric scale and nibble sign, and the code of NaN."""
@@ -60,6 +61,9 @@ MUTANTS = {
     19: "AWQ scales not normalised by the geometric mean",
     20: "clip search shrinks only the upper end",
     21: "AWQ activations multiplied by s",
+    22: "linear drops the last input channel",
+    23: "linear error scale sums signed terms",
+    24: "dequant truncates to bf16",
 }
 
 
